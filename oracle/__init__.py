@@ -1,0 +1,136 @@
+"""fp64 CPU oracle for exact scaled dot-product attention.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` use this module; the CUDA library never imports,
+links or calls it, and it never imports the CUDA library.
+
+The arithmetic lives in ``oracle.c`` (plain C, IEEE double, libm exp/log); this
+file only builds that shared object with gcc and marshals numpy/torch arrays
+into it.  It follows the three steps of standard attention named on the
+grasp.study lesson "The Computational Steps of Standard Self-Attention"
+(scores, row softmax, weighted sum of values) plus the log-sum-exp of each row.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_CFLAGS = ["-O2", "-fPIC", "-shared", "-std=c11", "-Wall", "-Wextra",
+           "-ffp-contract=off", "-pthread"]
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc); returns the path."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        for name, elem in (("oracle_attn_bf16", ctypes.c_void_p),
+                           ("oracle_attn_f64", ctypes.c_void_p)):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [elem, elem, elem, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                           ctypes.c_int, i64p, ctypes.c_int64, f64p, f64p,
+                           ctypes.c_int]
+        lib.oracle_probs_f64.restype = ctypes.c_int
+        lib.oracle_probs_f64.argtypes = [f64p, f64p, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_double, ctypes.c_int,
+                                         ctypes.c_int, f64p]
+        lib.oracle_default_threads.restype = ctypes.c_int
+        lib.oracle_default_threads.argtypes = []
+        _lib = lib
+        return lib
+
+
+def default_threads() -> int:
+    """Number of host threads the oracle uses when not told otherwise."""
+    return int(_load().oracle_default_threads())
+
+
+def all_rows(BH: int, N: int) -> np.ndarray:
+    """Every (bh, i) pair, shape [BH*N, 2] int64."""
+    bh = np.repeat(np.arange(BH, dtype=np.int64), N)
+    i = np.tile(np.arange(N, dtype=np.int64), BH)
+    return np.stack([bh, i], axis=1)
+
+
+def _as_bf16_bits(t) -> np.ndarray:
+    """torch bf16 tensor (any device) -> contiguous numpy uint16 bit patterns."""
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16:
+        raise TypeError("bf16 entry expects torch.bfloat16 tensors")
+    return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def attention(q, k, v, scale: float, causal: bool, rows=None, nthreads: int = 0):
+    """Exact attention rows in fp64.
+
+    q, k, v: [B, H, N, d], either torch.bfloat16 tensors (the bf16 values are
+    widened exactly) or float64 numpy arrays. rows: int64 array [R, 2] of
+    (bh, i) pairs with bh = b*H + h, or None for every row.
+    Returns (o [R, d] float64, lse [R] float64); lse is a natural logarithm.
+    """
+    lib = _load()
+    if isinstance(q, np.ndarray):
+        qa, ka, va = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+        fn = lib.oracle_attn_f64
+    else:
+        qa, ka, va = (_as_bf16_bits(x) for x in (q, k, v))
+        fn = lib.oracle_attn_bf16
+    if qa.ndim != 4 or ka.shape != qa.shape or va.shape != qa.shape:
+        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    B, H, N, d = (int(s) for s in qa.shape)
+    if rows is None:
+        rows = all_rows(B * H, N)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+    R = rows.shape[0]
+    o = np.zeros((R, d), dtype=np.float64)
+    lse = np.zeros((R,), dtype=np.float64)
+    st = fn(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, B, H, N, d,
+            float(scale), int(bool(causal)),
+            rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
+            o.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+            lse.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), int(nthreads))
+    if st != 0:
+        raise RuntimeError(f"oracle failed with status {st}")
+    return o, lse
+
+
+def probs_row(q: np.ndarray, k: np.ndarray, scale: float, causal: bool, i: int):
+    """Probability row p[0..N-1] of query i for one head (q, k: [N, d] float64)."""
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    N, d = q.shape
+    p = np.zeros((N,), dtype=np.float64)
+    f64p = ctypes.POINTER(ctypes.c_double)
+    st = lib.oracle_probs_f64(q.ctypes.data_as(f64p), k.ctypes.data_as(f64p), N, d,
+                              float(scale), int(bool(causal)), int(i),
+                              p.ctypes.data_as(f64p))
+    if st != 0:
+        raise RuntimeError(f"oracle_probs_f64 failed with status {st}")
+    return p

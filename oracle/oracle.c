@@ -1,0 +1,245 @@
+/*
+ * Exact scaled dot-product attention, fp64, on the CPU.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the oracle that the CUDA library is
+ * checked against. Only the tests, the smoke check and the CPU-baseline leg
+ * of the benchmark may load it; the product path never does. It shares no
+ * code, header, table or constant with the CUDA sources.
+ *
+ * What it computes, per (batch*head bh, query row i), follows the three steps
+ * of the standard attention computation as the pages describe them
+ * ("The Computational Steps of Standard Self-Attention", grasp.study lesson;
+ * and the boundary-crossing walk-through on "Attention Is Memory-Bound, and
+ * Nobody Noticed for Five Years", anylearn.cc):
+ *
+ *   1. scores      s_j = scale * sum_k q[i,k] * K[j,k]          for j in J(i)
+ *   2. softmax     p_j = exp(s_j - m) / l,  m = max_j s_j,  l = sum_j exp(s_j - m)
+ *   3. output      o[i,:] = sum_j p_j * V[j,:]
+ *
+ * plus the per-row log-sum-exp lse_i = m + ln(l) (natural logarithm).
+ *
+ * J(i) = {0..N-1}, or {0..i} when causal (key j allowed iff j <= i). Masked
+ * keys are excluded from the softmax, which is what setting their logit to
+ * -inf before the softmax means. A causal row always has key j = i, so no row
+ * is empty; if a row were empty anyway the oracle writes o = 0, lse = -inf.
+ *
+ * The anylearn.cc page ("FlashAttention computes exactly the same function as
+ * standard attention ... to within floating point reassociation") is why the
+ * plain definition is the oracle for the fused kernel.
+ *
+ * Inputs are either bf16 bit patterns (converted exactly to double) or
+ * doubles. All arithmetic is IEEE double with libm exp/log; no reassociation,
+ * no fused multiply-add (built with -ffp-contract=off).
+ *
+ * Rows to evaluate are given as (bh, i) pairs so that a seeded sample of rows
+ * can be checked on large shapes; rows are grouped by head, each head's K and
+ * V are converted to double once, and the head's rows are split over threads.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+enum { IN_BF16 = 0, IN_F64 = 1 };
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+static double bf16_bits_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double load_elem(const void *base, int kind, int64_t idx) {
+    if (kind == IN_F64) return ((const double *)base)[idx];
+    return bf16_bits_to_double(((const uint16_t *)base)[idx]);
+}
+
+/* Step 1: the row of scores for query q (length d) against keys 0..nkeys-1. */
+static void scores_row(const double *q, const double *K, int nkeys, int d,
+                       double scale, double *s) {
+    for (int j = 0; j < nkeys; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += q[c] * K[(int64_t)j * d + c];
+        s[j] = scale * dot;
+    }
+}
+
+/* Step 2: softmax of s[0..n-1] in place; returns m and l through pointers. */
+static void softmax_row(double *s, int n, double *m_out, double *l_out) {
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (s[j] > m) m = s[j];
+    double l = 0.0;
+    for (int j = 0; j < n; ++j) {
+        s[j] = exp(s[j] - m);
+        l += s[j];
+    }
+    for (int j = 0; j < n; ++j) s[j] /= l;
+    *m_out = m;
+    *l_out = l;
+}
+
+/* Step 3: o = sum_j p_j * V[j,:]. */
+static void output_row(const double *p, const double *V, int n, int d, double *o) {
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (int j = 0; j < n; ++j)
+        for (int c = 0; c < d; ++c) o[c] += p[j] * V[(int64_t)j * d + c];
+}
+
+/* One query row of one head: steps 1-3 and the log-sum-exp. */
+static void attend_row(const double *q, const double *K, const double *V, int N,
+                       int d, double scale, int causal, int i, double *s_buf,
+                       double *o, double *lse) {
+    int nkeys = causal ? i + 1 : N;
+    if (nkeys > N) nkeys = N;
+    if (nkeys <= 0) {
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    double m, l;
+    scores_row(q, K, nkeys, d, scale, s_buf);
+    softmax_row(s_buf, nkeys, &m, &l);
+    output_row(s_buf, V, nkeys, d, o);
+    *lse = m + log(l);
+}
+
+typedef struct {
+    const void *q;
+    int kind;
+    const double *K, *V; /* this head, converted */
+    int64_t bh;
+    int N, d, causal;
+    double scale;
+    const int64_t *rows;  /* all (bh, i) pairs */
+    const int64_t *mine;  /* indices into rows[] for this head */
+    int64_t nmine;
+    int tid, nthreads;
+    double *o, *lse;
+    int ok;        /* set to 1 by run_job when its rows are done */
+    int joinable;  /* 1 if run on its own pthread */
+} job_t;
+
+static void *run_job(void *arg) {
+    job_t *jb = (job_t *)arg;
+    double *s = (double *)malloc(sizeof(double) * (size_t)jb->N);
+    double *qrow = (double *)malloc(sizeof(double) * (size_t)jb->d);
+    if (!s || !qrow) {
+        jb->ok = 0;
+        free(s);
+        free(qrow);
+        return NULL;
+    }
+    for (int64_t t = jb->tid; t < jb->nmine; t += jb->nthreads) {
+        int64_t r = jb->mine[t];
+        int i = (int)jb->rows[2 * r + 1];
+        int64_t qoff = (jb->bh * jb->N + i) * (int64_t)jb->d;
+        for (int c = 0; c < jb->d; ++c) qrow[c] = load_elem(jb->q, jb->kind, qoff + c);
+        attend_row(qrow, jb->K, jb->V, jb->N, jb->d, jb->scale, jb->causal, i, s,
+                   jb->o + r * (int64_t)jb->d, jb->lse + r);
+    }
+    free(s);
+    free(qrow);
+    jb->ok = 1;
+    return NULL;
+}
+
+int oracle_default_threads(void) {
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    return n > 0 ? (int)n : 1;
+}
+
+static int attend(const void *q, const void *k, const void *v, int kind, int B,
+                  int H, int N, int d, double scale, int causal,
+                  const int64_t *rows, int64_t nrows, double *o, double *lse,
+                  int nthreads) {
+    if (!q || !k || !v || !rows || !o || !lse) return -1;
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || nrows < 0) return -2;
+    if (!isfinite(scale)) return -3;
+    if (nthreads <= 0) nthreads = oracle_default_threads();
+    int64_t BH = (int64_t)B * H;
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (rows[2 * r] < 0 || rows[2 * r] >= BH) return -4;
+        if (rows[2 * r + 1] < 0 || rows[2 * r + 1] >= N) return -4;
+    }
+    int64_t head_elems = (int64_t)N * d;
+    double *K = (double *)malloc(sizeof(double) * (size_t)head_elems);
+    double *V = (double *)malloc(sizeof(double) * (size_t)head_elems);
+    int64_t *mine = (int64_t *)malloc(sizeof(int64_t) * (size_t)(nrows > 0 ? nrows : 1));
+    job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    int status = 0;
+    if (!K || !V || !mine || !jobs || !th) status = -5;
+
+    for (int64_t bh = 0; bh < BH && status == 0; ++bh) {
+        int64_t nmine = 0;
+        for (int64_t r = 0; r < nrows; ++r)
+            if (rows[2 * r] == bh) mine[nmine++] = r;
+        if (nmine == 0) continue;
+        int64_t base = bh * head_elems;
+        for (int64_t e = 0; e < head_elems; ++e) {
+            K[e] = load_elem(k, kind, base + e);
+            V[e] = load_elem(v, kind, base + e);
+        }
+        int nt = nmine < nthreads ? (int)nmine : nthreads;
+        for (int t = 0; t < nt; ++t) {
+            job_t jb = {q, kind, K, V, bh, N, d, causal, scale, rows, mine, nmine,
+                        t, nt, o, lse, 0, 0};
+            jobs[t] = jb;
+        }
+        /* A thread that cannot be created runs its share inline. */
+        for (int t = 1; t < nt; ++t) {
+            if (pthread_create(&th[t], NULL, run_job, &jobs[t]) == 0)
+                jobs[t].joinable = 1;
+            else
+                run_job(&jobs[t]);
+        }
+        run_job(&jobs[0]);
+        for (int t = 1; t < nt; ++t)
+            if (jobs[t].joinable) pthread_join(th[t], NULL);
+        for (int t = 0; t < nt; ++t)
+            if (!jobs[t].ok) status = -5;
+    }
+    free(K);
+    free(V);
+    free(mine);
+    free(jobs);
+    free(th);
+    return status;
+}
+
+/* q, k, v: bf16 bit patterns, [B, H, N, d] contiguous. rows: nrows (bh, i)
+ * pairs. o: [nrows, d] doubles; lse: [nrows] doubles. nthreads <= 0 means all
+ * online cores. Returns 0 on success, negative on bad arguments or failure. */
+int oracle_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     int B, int H, int N, int d, double scale, int causal,
+                     const int64_t *rows, int64_t nrows, double *o, double *lse,
+                     int nthreads) {
+    return attend(q, k, v, IN_BF16, B, H, N, d, scale, causal, rows, nrows, o,
+                  lse, nthreads);
+}
+
+/* Same as oracle_attn_bf16 with double inputs (values need not be bf16). */
+int oracle_attn_f64(const double *q, const double *k, const double *v, int B,
+                    int H, int N, int d, double scale, int causal,
+                    const int64_t *rows, int64_t nrows, double *o, double *lse,
+                    int nthreads) {
+    return attend(q, k, v, IN_F64, B, H, N, d, scale, causal, rows, nrows, o,
+                  lse, nthreads);
+}
+
+/* The probability row p[0..N-1] of query i for a single head (q: [N, d],
+ * k: [N, d] doubles); masked keys get p = 0. Steps 1-2 only. */
+int oracle_probs_f64(const double *q, const double *k, int N, int d,
+                     double scale, int causal, int i, double *p) {
+    if (!q || !k || !p || N <= 0 || d <= 0 || i < 0 || i >= N) return -1;
+    int nkeys = causal ? i + 1 : N;
+    double m, l;
+    for (int j = 0; j < N; ++j) p[j] = 0.0;
+    scores_row(q + (int64_t)i * d, k, nkeys, d, scale, p);
+    softmax_row(p, nkeys, &m, &l);
+    return 0;
+}

@@ -1,0 +1,208 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle.
+
+Each test pins a part of the oracle to something independent: closed forms
+derived by hand, invariants of the softmax definition, brute force through a
+library softmax on tiny inputs, and exact-representability arguments. A
+plausible slip in the oracle (a dropped scale, a mask off by one, a transposed
+operand, a wrong log base, a missing max subtraction) fails at least one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_125_b200.inputs import make_qkv
+
+RNG = np.random.default_rng(12345)
+
+
+def _rand(B, H, N, d, scale=1.0):
+    return (RNG.standard_normal((B, H, N, d)) * scale for _ in range(3))
+
+
+def _flat(o, B, H, N, d):
+    return o.reshape(B, H, N, d)
+
+
+def test_two_key_closed_form():
+    # d = 1, N = 2, q = 1, keys chosen so the logits are s = (0, ln 3):
+    # exp(s) = (1, 3), so p = (1/4, 3/4), o = p . v = 3/4 with v = (0, 1),
+    # and lse = ln(1 + 3) = ln 4.
+    scale = 0.37
+    q = np.array([1.0, 1.0]).reshape(1, 1, 2, 1)
+    k = np.array([0.0, math.log(3.0) / scale]).reshape(1, 1, 2, 1)
+    v = np.array([0.0, 1.0]).reshape(1, 1, 2, 1)
+    o, lse = oracle.attention(q, k, v, scale, causal=False)
+    assert abs(o[0, 0] - 0.75) < 1e-15 and abs(o[1, 0] - 0.75) < 1e-15
+    assert abs(lse[0] - math.log(4.0)) < 1e-15
+    # causal: row 0 sees key 0 only (o = v0 = 0, lse = s00 = 0); row 1 sees both.
+    o, lse = oracle.attention(q, k, v, scale, causal=True)
+    assert o[0, 0] == 0.0 and lse[0] == 0.0
+    assert abs(o[1, 0] - 0.75) < 1e-15 and abs(lse[1] - math.log(4.0)) < 1e-15
+
+
+def test_large_logits_stay_finite():
+    # logits (1000, 1000 + ln 3): a version without the max subtraction
+    # overflows exp(); the exact answer is the same as the two-key case shifted.
+    scale = 1.0
+    q = np.array([1.0, 1.0]).reshape(1, 1, 2, 1)
+    k = np.array([1000.0, 1000.0 + math.log(3.0)]).reshape(1, 1, 2, 1)
+    v = np.array([0.0, 1.0]).reshape(1, 1, 2, 1)
+    o, lse = oracle.attention(q, k, v, scale, causal=False)
+    assert abs(o[0, 0] - 0.75) < 1e-13
+    assert abs(lse[0] - (1000.0 + math.log(4.0))) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(1, 1), (2, 2), (5, 4), (16, 1), (13, 3)])
+def test_brute_force_vs_torch_softmax(N, d, causal):
+    # softmax(Q K^T * scale + mask) V through torch's own float64 softmax.
+    B, H = 2, 3
+    q, k, v = _rand(B, H, N, d)
+    scale = 0.7
+    o, lse = oracle.attention(q, k, v, scale, causal)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    logits = torch.einsum("bhid,bhjd->bhij", tq, tk) * scale
+    if causal:
+        mask = torch.ones(N, N, dtype=torch.bool).triu(1)
+        logits = logits.masked_fill(mask, float("-inf"))
+    ref = torch.softmax(logits, dim=-1) @ tv
+    ref_lse = torch.logsumexp(logits, dim=-1)
+    assert np.abs(o - ref.numpy().reshape(-1, d)).max() <= 1e-12
+    assert np.abs(lse - ref_lse.numpy().reshape(-1)).max() <= 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_scale_zero_is_mean_of_allowed_values(causal):
+    # scale = 0 makes every allowed logit 0: each allowed key gets 1/|J(i)|,
+    # so o_i = mean of v_0..v_i (causal) or of all v (non-causal) and
+    # lse_i = ln |J(i)|. A mask that is off by one changes both.
+    B, H, N, d = 1, 2, 9, 3
+    q, k, v = _rand(B, H, N, d)
+    o, lse = oracle.attention(q, k, v, 0.0, causal)
+    o = o.reshape(B, H, N, d)
+    lse = lse.reshape(B, H, N)
+    for h in range(H):
+        for i in range(N):
+            n = i + 1 if causal else N
+            assert np.abs(o[0, h, i] - v[0, h, :n].mean(axis=0)).max() < 1e-14
+            assert abs(lse[0, h, i] - math.log(n)) < 1e-14
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_values_give_constant_output(causal):
+    # each probability row sums to one, so V rows all equal to c give O = c;
+    # with V = 1 this is the row-sum invariant itself.
+    B, H, N, d = 2, 2, 17, 5
+    q, k, _ = _rand(B, H, N, d, 2.0)
+    c = RNG.standard_normal(d)
+    v = np.broadcast_to(c, (B, H, N, d)).copy()
+    o, _ = oracle.attention(q, k, v, 0.3, causal)
+    assert np.abs(o - c).max() < 1e-13
+    o1, _ = oracle.attention(q, k, np.ones_like(v), 0.3, causal)
+    assert np.abs(o1 - 1.0).max() < 1e-14
+
+
+def test_single_key():
+    # N = 1: the only probability is 1, o = v0, lse = scale * q0 . k0.
+    q, k, v = _rand(3, 2, 1, 6)
+    o, lse = oracle.attention(q, k, v, 0.25, causal=False)
+    assert np.abs(o - v.reshape(-1, 6)).max() == 0.0
+    want = 0.25 * np.einsum("bhid,bhid->bhi", q, k).reshape(-1)
+    assert np.abs(lse - want).max() < 1e-14
+
+
+def test_causal_first_row_is_first_value():
+    q, k, v = _rand(2, 2, 11, 4, 3.0)
+    rows = np.array([[bh, 0] for bh in range(4)], dtype=np.int64)
+    o, lse = oracle.attention(q, k, v, 0.5, True, rows=rows)
+    assert np.abs(o - v[:, :, 0, :].reshape(4, 4)).max() == 0.0
+    want = 0.5 * np.einsum("bhd,bhd->bh", q[:, :, 0], k[:, :, 0]).reshape(-1)
+    assert np.abs(lse - want).max() < 1e-14
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_per_row_logit_shift(causal):
+    # K' = K + 1 u^T adds scale * (q_i . u) to every logit of row i: the
+    # softmax is unchanged, lse shifts by exactly that amount.
+    B, H, N, d = 1, 2, 12, 4
+    q, k, v = _rand(B, H, N, d)
+    u = RNG.standard_normal(d)
+    scale = 0.6
+    o, lse = oracle.attention(q, k, v, scale, causal)
+    o2, lse2 = oracle.attention(q, k + u, v, scale, causal)
+    shift = scale * (q @ u).reshape(-1)
+    assert np.abs(o2 - o).max() < 1e-13
+    assert np.abs(lse2 - lse - shift).max() < 1e-12
+
+
+def test_key_permutation_invariance():
+    # non-causal attention does not depend on the order of the (key, value)
+    # pairs; a transposed or mis-indexed K or V breaks this.
+    B, H, N, d = 1, 1, 10, 3
+    q, k, v = _rand(B, H, N, d)
+    perm = RNG.permutation(N)
+    o, lse = oracle.attention(q, k, v, 0.8, False)
+    o2, lse2 = oracle.attention(q, k[:, :, perm], v[:, :, perm], 0.8, False)
+    assert np.abs(o - o2).max() < 1e-14 and np.abs(lse - lse2).max() < 1e-14
+
+
+def test_asymmetric_scores_orientation():
+    # s_ij = q_i . k_j, not q_j . k_i: with one query row much longer than the
+    # keys, swapping the operands gives a different answer. Keys are 1-hot so
+    # s_ij = q_i[j]; row 0 picks key 2 (logit 50), row 1 picks key 0.
+    q = np.zeros((1, 1, 3, 3)); k = np.eye(3).reshape(1, 1, 3, 3)
+    q[0, 0, 0] = [0.0, 0.0, 50.0]
+    q[0, 0, 1] = [50.0, 0.0, 0.0]
+    v = np.array([[1.0, 0, 0], [0, 1.0, 0], [0, 0, 1.0]]).reshape(1, 1, 3, 3)
+    o, _ = oracle.attention(q, k, v, 1.0, False)
+    assert o[0, 2] > 1 - 1e-15 and o[1, 0] > 1 - 1e-15
+    assert o[0, 0] < 1e-20 and o[1, 2] < 1e-20
+    # row 2 has q = 0: every logit is 0, uniform weights
+    assert np.abs(o[2] - 1.0 / 3.0).max() < 1e-15
+
+
+def test_probability_row_properties():
+    N, d = 14, 5
+    q = RNG.standard_normal((N, d))
+    k = RNG.standard_normal((N, d))
+    for causal in (False, True):
+        for i in (0, 5, N - 1):
+            p = oracle.probs_row(q, k, 0.4, causal, i)
+            assert abs(p.sum() - 1.0) < 1e-15
+            assert (p >= 0).all()
+            if causal:
+                assert (p[i + 1:] == 0).all() and (p[: i + 1] > 0).all()
+            ref = torch.softmax(torch.from_numpy(q[i] @ k[: (i + 1 if causal else N)].T * 0.4), 0)
+            assert np.abs(p[: len(ref)] - ref.numpy()).max() < 1e-15
+
+
+def test_bf16_entry_widens_exactly():
+    # The bf16 entry must give bit-identical results to the f64 entry fed
+    # the same values (bf16 -> double is exact).
+    q, k, v = make_qkv(2, 2, 37, 8, seed=7)
+    o, lse = oracle.attention(q, k, v, 0.35, True)
+    o2, lse2 = oracle.attention(q.double().numpy(), k.double().numpy(),
+                                v.double().numpy(), 0.35, True)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def test_sampled_rows_equal_full_rows_and_threads_agree():
+    q, k, v = make_qkv(2, 3, 50, 8, seed=9)
+    o_all, lse_all = oracle.attention(q, k, v, 0.3, True, nthreads=1)
+    rows = np.array([[5, 49], [0, 0], [3, 17], [5, 3]], dtype=np.int64)
+    o, lse = oracle.attention(q, k, v, 0.3, True, rows=rows, nthreads=4)
+    flat = rows[:, 0] * 50 + rows[:, 1]
+    assert np.array_equal(o, o_all[flat]) and np.array_equal(lse, lse_all[flat])
+    o_mt, _ = oracle.attention(q, k, v, 0.3, True, nthreads=7)
+    assert np.array_equal(o_mt, o_all)
+
+
+def test_rejects_bad_rows():
+    q, k, v = make_qkv(1, 1, 4, 2, seed=1)
+    with pytest.raises(RuntimeError):
+        oracle.attention(q, k, v, 1.0, False, rows=np.array([[0, 4]]))
+    with pytest.raises(RuntimeError):
+        oracle.attention(q, k, v, float("nan"), False)
