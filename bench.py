@@ -1,0 +1,474 @@
+"""Throughput of the fused exact-attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is one attn_fwd over the whole workload: B=8, H=32, N=8192, d=128,
+causal, bf16 Q/K/V drawn N(0,1) from a fixed seed (the batch/head/length of
+the score-matrix memory example on the anylearn.cc page "Attention Is
+Memory-Bound, and Nobody Noticed for Five Years"). Metric: TFLOP/s with
+4*B*H*N^2*d FLOPs per step, halved for causal.
+
+With N > 1 (torchrun, one process per GPU) each rank runs its own copy of the
+workload: the (batch, head) units are independent, so there is no
+data-path collective ("weak" scaling); the barrier and the max-over-ranks of
+the device time are measurement only.
+
+Prints one JSON line on rank 0. `--impl reference` times the fp64 CPU oracle
+on a bounded sample of the same workload instead (CPU only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "long_8192_causal"
+METRIC = "attn fwd TFLOP/s (causal-adjusted) and % of B200 dense BF16 peak"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_attn_fwd_long_8192_causal.txt")
+KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_125_b200", "csrc", "fused_fwd.cu")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=WORKLOAD)
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-naive", action="store_true", help="skip the unfused traffic line")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0,
+                   help="target CPU time of the oracle sample")
+    return p.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(path=KERNEL_SOURCE) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+    or None when the summary is missing or was taken on another kernel source."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    fields = {}
+    for line in open(PROFILE_SUMMARY):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("kernel_source_sha256_16") != source_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch_full_workload"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        return summarize_clocks(rows)
+
+
+def summarize_clocks(rows):
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+    def num(x):
+        try:
+            return float(x)
+        except ValueError:
+            return None
+    sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+    mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = set()
+    for r in rows:
+        for name, val in zip(names, r[5:9]):
+            if val.strip().lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(mx) if mx else None,
+            "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+# ------------------------------------------------------------ oracle (CPU)
+def cpu_oracle_sample(w, target_seconds: float):
+    """Times the fp64 oracle on a bounded, seeded sample of the workload's rows.
+    Returns (tflops, seconds, rows, cores, sample description)."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_125_b200.inputs import make_qkv
+
+    # the oracle needs only the sampled heads: draw a 2-head slice with the
+    # workload's distribution (same per-row work as any head of the workload)
+    q, k, v = make_qkv(1, 2, w.N, w.d, w.seed, w.dist)
+    cores = oracle.default_threads()
+    rng = np.random.default_rng(w.seed)
+
+    def rows_for(n):
+        i = np.sort(rng.choice(w.N, size=n, replace=False))
+        bh = np.arange(n) % 2
+        return np.stack([bh, i], 1).astype(np.int64)
+
+    def flops(rows):
+        keys = (rows[:, 1] + 1) if w.causal else np.full(len(rows), w.N)
+        return float(4.0 * w.d * keys.sum())
+
+    probe = rows_for(max(cores, 16))
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, w.scale, w.causal, rows=probe)
+    dt = time.perf_counter() - t0
+    per_row = dt / len(probe)
+    n = int(min(w.N, max(len(probe), target_seconds / max(per_row, 1e-9))))
+    rows = rows_for(n)
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, w.scale, w.causal, rows=rows)
+    secs = time.perf_counter() - t0
+    desc = (f"{n} seeded query rows of {w.name} (B=1 slice of 2 heads, same N, d, "
+            f"causal={w.causal}, distribution {w.dist}); FLOPs counted 4*d*|allowed keys| per row")
+    return flops(rows) / secs / 1e12, secs, n, cores, desc
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from exact_attention_125_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    per_step = []
+    total_rows = 0
+    cores = 0
+    desc = ""
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, 1.0)
+    for _ in range(args.steps):
+        tf, secs, n, cores, desc = cpu_oracle_sample(w, max(1.0, args.cpu_seconds / max(args.steps, 1)))
+        per_step.append((tf, secs))
+        total_rows += n
+    tflops = statistics.median(t for t, _ in per_step)
+    ms = statistics.median(s for _, s in per_step) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "sample": "bounded row sample per step"},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------- GPU bench
+def run_ours(args):
+    import torch
+
+    import exact_attention_125_b200 as ea
+    from exact_attention_125_b200 import costs
+    from exact_attention_125_b200.inputs import WORKLOADS, make_workload
+
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        if not (world == 1 and args.gpus == 1):
+            raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch with torchrun")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    w = WORKLOADS[args.workload]
+    peaks, peaks_kind = load_peaks()
+
+    # seeded inputs (per-rank seed offset: each rank owns a different batch)
+    qh, kh, vh = make_workload(w) if rank == 0 else _rank_inputs(w, rank)
+    q, k, v = (t.to(device) for t in (qh, kh, vh))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    flops = costs.attn_flops(w.B, w.H, w.N, w.d, w.causal)
+
+    def step():
+        ea.attn_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if ea.last_device_error() != 0:
+        raise SystemExit("device watchdog fired during warm-up")
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(dist)
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(dist)
+    ms_local = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_local, dist, device)
+    if ea.last_device_error() != 0:
+        raise SystemExit("device watchdog fired in the timed region")
+    ms_step = ms_total / args.steps
+    value = flops * world * args.steps / (ms_total * 1e-3) / 1e12
+    launch_tflops = flops / (ms_local / args.steps * 1e-3) / 1e12
+    clock_info = clocks.summary()
+
+    e2e = e2e_through_abi(args, w, qh, kh, vh, device, dist, flops, world)
+    naive = None if args.no_naive else naive_line(w, device, peaks)
+
+    peak = float(peaks["bf16_tflops"])
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "per_rank": "one full copy of the workload",
+                   "l2": "inputs larger than L2 (Q, K, V 1.5 GiB per step)",
+                   "parallelism": f"replicas x{world}"},
+        "pct_of_peak": {
+            f"of_{peaks_kind}_burst_{peak:g}": 100.0 * launch_tflops / peak,
+            f"of_{peaks_kind}_sustained_{float(peaks['bf16_tflops_sustained']):g}":
+                100.0 * launch_tflops / float(peaks["bf16_tflops_sustained"]),
+            "of_spec_2250": 100.0 * launch_tflops / 2250.0,
+        },
+        "roofline": {
+            "bound": "tensor",
+            "achieved": launch_tflops,
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": launch_tflops / peak,
+            "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peaks_kind}, burst)",
+            "traffic": profiled_traffic(),
+            "algorithmic_bytes": costs.fused_bytes(w.B, w.H, w.N, w.d),
+            "kernel": "fused_attn_fwd_kernel<128>",
+        },
+        "clocks": {k: clock_info[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+    }
+    if naive is not None:
+        line["naive"] = naive
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, secs, n, cores, desc = cpu_oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def _rank_inputs(w, rank):
+    from exact_attention_125_b200.inputs import make_qkv
+    return make_qkv(w.B, w.H, w.N, w.d, w.seed + 7919 * rank, w.dist)
+
+
+def e2e_through_abi(args, w, qh, kh, vh, device, dist, flops, world):
+    """Same metric through the C ABI with host buffers: every step copies Q, K, V
+    from pinned host memory, runs attn_fwd, and copies O and lse back."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    q_h, k_h, v_h = (t.pin_memory() for t in (qh, kh, vh))
+    o_h = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    l_h = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    q, k, v = (torch.empty_like(t, device=device) for t in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    h = stream.cuda_stream
+
+    def step():
+        for dst, src in ((q, q_h), (k, k_h), (v, v_h)):
+            dst.copy_(src, non_blocking=True)
+        st = ea.abi.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal), h)
+        if st != 0:
+            raise ea.AttnError(st, "attn_fwd")
+        o_h.copy_(o, non_blocking=True)
+        l_h.copy_(lse, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    start.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(start.elapsed_time(end), dist, device)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = o_h.numel() * o_h.element_size() + l_h.numel() * l_h.element_size()
+    return {"value": flops * world * args.e2e_steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / args.e2e_steps, "steps": args.e2e_steps,
+            "path": "pinned host -> device copy, attn_fwd via the C ABI, device -> pinned host"}
+
+
+def naive_line(w, device, peaks, steps=2):
+    """The unfused path on the same workload, heads in groups so the S/P
+    workspace stays bounded; reported as achieved HBM GB/s of its algorithmic
+    traffic (four crossings of S and P plus Q, K, V, O, lse)."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    from exact_attention_125_b200 import costs
+    BH = w.B * w.H
+    per_head_ws = ea.naive_workspace_bytes(1, 1, w.N)
+    free, _ = torch.cuda.mem_get_info(device)
+    group = max(1, min(BH, int(min(free * 0.6, 40e9) // per_head_ws)))
+    while BH % group:
+        group -= 1
+    q = torch.randn((BH, w.N, w.d), device=device, dtype=torch.bfloat16)
+    k, v = torch.randn_like(q), torch.randn_like(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((BH, w.N), dtype=torch.float32, device=device)
+    ws = torch.empty((per_head_ws * group,), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for g0 in range(0, BH, group):
+            ea.attn_fwd_naive(q[g0:g0 + group].unsqueeze(0), k[g0:g0 + group].unsqueeze(0),
+                              v[g0:g0 + group].unsqueeze(0), o[g0:g0 + group].unsqueeze(0),
+                              lse[g0:g0 + group].unsqueeze(0), scale=w.scale, causal=w.causal,
+                              workspace=ws, stream=stream)
+
+    step()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end) / steps
+    nbytes = costs.naive_bytes(w.B, w.H, w.N, w.d)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del ws
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+            "hbm_peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
+            "tflops": costs.attn_flops(w.B, w.H, w.N, w.d, w.causal) / (ms * 1e-3) / 1e12,
+            "head_group": group, "launches_per_step": 3 * (BH // group)}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,173 @@
+"""B200-native (sm_100a) exact attention forward.
+
+Python binding of the C ABI in include/attn.h (libattn_b200.so, built in this
+directory). This module only marshals arguments: every step of the attention
+computation runs in the library's CUDA kernels. There is no CPU fallback; if
+the library is missing, every call raises.
+
+The torch-facing helpers take CUDA bf16 tensors of shape [B, H, N, d] and
+allocate outputs with torch when none are given (the library never allocates).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+__all__ = [
+    "AttnError", "lib", "attn_fwd", "attn_fwd_naive", "naive_workspace_bytes",
+    "last_device_error", "status_string", "selftest_wait_timeout", "abi",
+]
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+ATTN_OK = 0
+STATUS = {
+    0: "ATTN_OK", -1: "ATTN_ERR_NULL", -2: "ATTN_ERR_SHAPE", -3: "ATTN_ERR_HEADDIM",
+    -4: "ATTN_ERR_ALIGN", -5: "ATTN_ERR_SCALE", -6: "ATTN_ERR_CAUSAL",
+    -7: "ATTN_ERR_WORKSPACE", -8: "ATTN_ERR_LAUNCH", -9: "ATTN_ERR_UNSUPPORTED_DEVICE",
+    -10: "ATTN_ERR_TIMEOUT", -11: "ATTN_ERR_CUDA",
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libattn_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"libattn_b200.so not found at {_LIB_PATH}; build it with "
+                "`python -m exact_attention_125_b200._build` (no CPU fallback exists)")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.attn_fwd.restype = i
+        L.attn_fwd_naive_workspace_bytes.argtypes = [i, i, i]
+        L.attn_fwd_naive_workspace_bytes.restype = sz
+        L.attn_fwd_naive.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+        L.attn_fwd_naive.restype = i
+        L.attn_last_device_error.argtypes = [vp]
+        L.attn_last_device_error.restype = i
+        L.attn_status_string.argtypes = [i]
+        L.attn_status_string.restype = ctypes.c_char_p
+        L.attn_selftest_wait_timeout.argtypes = [i, vp]
+        L.attn_selftest_wait_timeout.restype = i
+        _lib = L
+        return L
+
+
+class abi:
+    """The C entry points with raw pointers and sizes, same names as attn.h."""
+
+    @staticmethod
+    def attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream) -> int:
+        return lib().attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream)
+
+    @staticmethod
+    def attn_fwd_naive(q, k, v, o, lse, B, H, N, d, scale, causal, ws, ws_bytes, stream) -> int:
+        return lib().attn_fwd_naive(q, k, v, o, lse, B, H, N, d, scale, causal, ws, ws_bytes,
+                                    stream)
+
+    @staticmethod
+    def attn_fwd_naive_workspace_bytes(B, H, N) -> int:
+        return int(lib().attn_fwd_naive_workspace_bytes(B, H, N))
+
+    @staticmethod
+    def attn_last_device_error(stream) -> int:
+        return lib().attn_last_device_error(stream)
+
+    @staticmethod
+    def attn_status_string(status) -> str:
+        return lib().attn_status_string(status).decode()
+
+    @staticmethod
+    def attn_selftest_wait_timeout(limit_ms, stream) -> int:
+        return lib().attn_selftest_wait_timeout(limit_ms, stream)
+
+
+def status_string(status: int) -> str:
+    return abi.attn_status_string(status)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_qkv(q, k, v):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous bf16 [B, H, N, d] tensor")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+    return tuple(int(s) for s in q.shape)
+
+
+def _outputs(q, o, lse):
+    import torch
+    B, H, N, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    return o, lse
+
+
+def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
+    """Fused forward. Returns (o, lse); o is bf16 [B,H,N,d], lse fp32 [B,H,N]."""
+    B, H, N, d = _check_qkv(q, k, v)
+    o, lse = _outputs(q, o, lse)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = abi.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def naive_workspace_bytes(B: int, H: int, N: int) -> int:
+    return abi.attn_fwd_naive_workspace_bytes(B, H, N)
+
+
+def attn_fwd_naive(q, k, v, o=None, lse=None, scale=None, causal=False, workspace=None,
+                   stream=None):
+    """Unfused three-kernel forward (S and P in HBM). Returns (o, lse)."""
+    import torch
+    B, H, N, d = _check_qkv(q, k, v)
+    o, lse = _outputs(q, o, lse)
+    need = naive_workspace_bytes(B, H, N)
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = abi.attn_fwd_naive(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                            lse.data_ptr(), B, H, N, d, scale, int(bool(causal)),
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_naive")
+    return o, lse
+
+
+def last_device_error(stream=None) -> int:
+    """Reads and clears the device error word (synchronises the stream)."""
+    return abi.attn_last_device_error(_stream_handle(stream))
+
+
+def selftest_wait_timeout(limit_ms: int, stream=None) -> int:
+    return abi.attn_selftest_wait_timeout(int(limit_ms), _stream_handle(stream))

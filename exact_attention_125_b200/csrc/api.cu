@@ -1,0 +1,133 @@
+// api.cu - the C ABI of libattn_b200.so (declared in include/attn.h):
+// argument validation, device check, dispatch to the fused or naive path.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "internal.h"
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int validate(const void* q, const void* k, const void* v, const void* o, const float* lse, int B,
+             int H, int N, int d, float scale, int causal) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+  if (B < 1 || H < 1 || N < 1) return ATTN_ERR_SHAPE;
+  if (static_cast<long long>(B) * H * N > INT_MAX) return ATTN_ERR_SHAPE;
+  if (d != 64 && d != 128) return ATTN_ERR_HEADDIM;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4))
+    return ATTN_ERR_ALIGN;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_SCALE;
+  if (causal != 0 && causal != 1) return ATTN_ERR_CAUSAL;
+  return ATTN_OK;
+}
+
+// sm_100 check of the current device, cached per device ordinal.
+int check_device() {
+  static int state[64] = {0};  // 0 unknown, 1 ok, -1 unsupported
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return ATTN_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (state[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    state[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return state[dev] == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED_DEVICE;
+}
+
+attn::AttnArgs pack(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int N, int d, float scale, int causal) {
+  attn::AttnArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.scale = scale;
+  a.causal = causal;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int N, int d, float scale, int causal, attn_stream_t stream) {
+  int st = validate(q, k, v, o, lse, B, H, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if ((st = check_device()) != ATTN_OK) return st;
+  return attn::launch_fused(pack(q, k, v, o, lse, B, H, N, d, scale, causal),
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t attn_fwd_naive_workspace_bytes(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  const unsigned long long bh = static_cast<unsigned long long>(B) * H;
+  const unsigned long long nn = static_cast<unsigned long long>(N) * N;
+  if (bh > (1ull << 31) || nn > (1ull << 40)) return 0;
+  const unsigned long long elems = bh * nn;
+  if (elems > (~0ull) / 4) return 0;
+  return static_cast<size_t>(elems * 4ull);  // S and P, bf16 each
+}
+
+int attn_fwd_naive(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                   attn_stream_t stream) {
+  int st = validate(q, k, v, o, lse, B, H, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (N > 32768 || static_cast<long long>(B) * H > 65535) return ATTN_ERR_SHAPE;
+  if (!workspace) return ATTN_ERR_NULL;
+  if (!aligned(workspace, 16)) return ATTN_ERR_ALIGN;
+  const size_t need = attn_fwd_naive_workspace_bytes(B, H, N);
+  if (need == 0 || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if ((st = check_device()) != ATTN_OK) return st;
+  return attn::launch_naive(pack(q, k, v, o, lse, B, H, N, d, scale, causal), workspace,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_last_device_error(attn_stream_t stream) {
+  return attn::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_selftest_wait_timeout(int limit_ms, attn_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 5000) return ATTN_ERR_SHAPE;
+  int st = check_device();
+  if (st != ATTN_OK) return st;
+  return attn::launch_wait_timeout_selftest(limit_ms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_NULL: return "ATTN_ERR_NULL: a required pointer is NULL";
+    case ATTN_ERR_SHAPE: return "ATTN_ERR_SHAPE: B, H or N out of range";
+    case ATTN_ERR_HEADDIM: return "ATTN_ERR_HEADDIM: d must be 64 or 128";
+    case ATTN_ERR_ALIGN: return "ATTN_ERR_ALIGN: pointer misaligned";
+    case ATTN_ERR_SCALE: return "ATTN_ERR_SCALE: scale must be finite and > 0";
+    case ATTN_ERR_CAUSAL: return "ATTN_ERR_CAUSAL: causal must be 0 or 1";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: workspace too small";
+    case ATTN_ERR_LAUNCH: return "ATTN_ERR_LAUNCH: kernel launch failed";
+    case ATTN_ERR_UNSUPPORTED_DEVICE: return "ATTN_ERR_UNSUPPORTED_DEVICE: needs an sm_100 GPU";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT: a device-side bounded wait ran out";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA runtime call failed";
+    default: return "unknown attn status";
+  }
+}
+
+}  // extern "C"

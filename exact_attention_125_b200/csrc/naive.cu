@@ -1,0 +1,398 @@
+// naive.cu - the deliberately unfused standard attention path.
+//
+// Three kernels, each reading its input from HBM and writing its output back,
+// as the anylearn.cc page "Attention Is Memory-Bound, and Nobody Noticed for
+// Five Years" traces the textbook implementation:
+//   1. scores:  S = scale * Q K^T (bf16, causally masked entries = -inf)  -> HBM
+//   2. softmax: P = softmax(S) row by row (fp32 math, bf16 out), lse (fp32) -> HBM
+//   3. values:  O = P V (fp32 accumulate, bf16 out)                       -> HBM
+// The N x N matrices S and P each cross the HBM boundary twice. This path is
+// a measuring stick for that traffic, not a product path: its two matrix
+// products use warp-level mma.sync tensor-core instructions so that it is
+// bound by memory, as the pages say it is, rather than by scalar arithmetic.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/attn.h"
+#include "internal.h"
+
+namespace attn {
+namespace {
+
+constexpr int kT = 128;          // output tile rows/cols
+constexpr int kChunk = 64;       // keys per step of the P.V kernel
+constexpr uint16_t kBf16NegInf = 0xFF80u;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// c += a * b for one m16n8k16 bf16 tile, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Eight consecutive bf16 of a row with `valid` readable elements starting at
+// `p`; vector load when allowed, else element by element with zero fill.
+__device__ __forceinline__ uint4 load8(const uint16_t* p, int valid, bool vec_ok) {
+  if (vec_ok && valid >= 8) return *reinterpret_cast<const uint4*>(p);
+  uint16_t e[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) e[u] = (u < valid) ? p[u] : uint16_t(0);
+  return make_uint4(e[0] | (uint32_t(e[1]) << 16), e[2] | (uint32_t(e[3]) << 16),
+                    e[4] | (uint32_t(e[5]) << 16), e[6] | (uint32_t(e[7]) << 16));
+}
+
+// ----------------------------------------------------------------- scores
+// One 128 x 128 tile of S per CTA (8 warps as 2 x 4, each 64 x 32).
+template <int D>
+__global__ void __launch_bounds__(256) naive_scores_kernel(const uint16_t* __restrict__ q,
+                                                           const uint16_t* __restrict__ k,
+                                                           uint16_t* __restrict__ S, int N,
+                                                           float scale, int causal) {
+  constexpr int LD = D + 8;       // padded smem row (elements)
+  constexpr int LDS = kT + 8;     // staging row
+  extern __shared__ __align__(16) uint16_t sm[];
+  uint16_t* Qs = sm;
+  uint16_t* Ks = sm + kT * LD;
+  const int c0 = blockIdx.x * kT, r0 = blockIdx.y * kT, bh = blockIdx.z;
+  const size_t head = static_cast<size_t>(bh) * N;
+  uint16_t* Sh = S + head * N;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const bool vec_ok = (N % 8) == 0;
+
+  if (causal && c0 > r0 + kT - 1) {  // tile entirely above the diagonal
+    for (int e = tid; e < kT * kT; e += 256) {
+      const int r = r0 + e / kT, c = c0 + e % kT;
+      if (r < N && c < N) Sh[static_cast<size_t>(r) * N + c] = kBf16NegInf;
+    }
+    return;
+  }
+
+  for (int e = tid; e < kT * (D / 8); e += 256) {
+    const int r = e / (D / 8), cv = (e % (D / 8)) * 8;
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(Qs + r * LD + cv) =
+        (r0 + r < N) ? *reinterpret_cast<const uint4*>(q + (head + r0 + r) * D + cv) : zero;
+    *reinterpret_cast<uint4*>(Ks + r * LD + cv) =
+        (c0 + r < N) ? *reinterpret_cast<const uint4*>(k + (head + c0 + r) * D + cv) : zero;
+  }
+  __syncthreads();
+
+  const int wm = warp / 4, wn = warp % 4;
+  float acc[4][4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[i][j][u] = 0.0f;
+
+#pragma unroll
+  for (int kk = 0; kk < D; kk += 16) {
+    uint32_t a[4][4], b[4][2];
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+      ldsm_x4(smem_addr(Qs + (wm * 64 + mi * 16 + (lane % 16)) * LD + kk + (lane / 16) * 8), a[mi]);
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni)
+      ldsm_x2(smem_addr(Ks + (wn * 32 + ni * 8 + (lane % 8)) * LD + kk + ((lane / 8) % 2) * 8),
+              b[ni]);
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < 4; ++ni) mma16816(acc[mi][ni], a[mi], b[ni][0], b[ni][1]);
+  }
+  __syncthreads();
+
+  // scale, mask, round to bf16, stage the tile in shared memory
+  uint16_t* St = sm;
+  const float ninf = __uint_as_float(0xff800000u);
+#pragma unroll
+  for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = wm * 64 + mi * 16 + lane / 4 + 8 * h;
+        const int c = wn * 32 + ni * 8 + (lane % 4) * 2;
+        float v0 = acc[mi][ni][2 * h] * scale, v1 = acc[mi][ni][2 * h + 1] * scale;
+        if (causal) {
+          if (c0 + c > r0 + r) v0 = ninf;
+          if (c0 + c + 1 > r0 + r) v1 = ninf;
+        }
+        *reinterpret_cast<uint32_t*>(St + r * LDS + c) = bf16x2_bits(v0, v1);
+      }
+  __syncthreads();
+
+  if (vec_ok && r0 + kT <= N && c0 + kT <= N) {
+    for (int e = tid; e < kT * (kT / 8); e += 256) {
+      const int r = e / (kT / 8), cv = (e % (kT / 8)) * 8;
+      *reinterpret_cast<uint4*>(Sh + static_cast<size_t>(r0 + r) * N + c0 + cv) =
+          *reinterpret_cast<const uint4*>(St + r * LDS + cv);
+    }
+  } else {
+    for (int e = tid; e < kT * kT; e += 256) {
+      const int r = e / kT, c = e % kT;
+      if (r0 + r < N && c0 + c < N) Sh[static_cast<size_t>(r0 + r) * N + c0 + c] = St[r * LDS + c];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- softmax
+// One CTA per row of S; each thread keeps EPT elements of the row in registers
+// so S is read once and P written once.
+template <int EPT>
+__global__ void __launch_bounds__(512) naive_softmax_kernel(const uint16_t* __restrict__ S, uint16_t* __restrict__ P,
+                                     float* __restrict__ lse, int N) {
+  __shared__ float red[32];
+  const size_t row = blockIdx.x;
+  const uint16_t* srow = S + row * N;
+  uint16_t* prow = P + row * N;
+  const int T = blockDim.x, tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int nwarps = T / 32;
+  const bool vec = (N % 8) == 0;
+  float x[EPT];
+  const float ninf = __uint_as_float(0xff800000u);
+
+  if (vec) {
+#pragma unroll
+    for (int i = 0; i < EPT / 8; ++i) {
+      const int e = (tid + i * T) * 8;
+      uint4 w = make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+      if (e < N) w = *reinterpret_cast<const uint4*>(srow + e);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        x[i * 8 + 2 * u] = __uint_as_float(ws[u] << 16);
+        x[i * 8 + 2 * u + 1] = __uint_as_float(ws[u] & 0xffff0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      const int e = tid + i * T;
+      x[i] = (e < N) ? __uint_as_float(uint32_t(srow[e]) << 16) : ninf;
+    }
+  }
+
+  float m = ninf;
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) m = fmaxf(m, x[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  m = ninf;
+  for (int w = 0; w < nwarps; ++w) m = fmaxf(m, red[w]);
+  __syncthreads();
+
+  const float l2e = 1.4426950408889634f;
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) {
+    x[i] = exp2f((x[i] - m) * l2e);
+    s += x[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red[warp] = s;
+  __syncthreads();
+  s = 0.0f;
+  for (int w = 0; w < nwarps; ++w) s += red[w];
+  const float inv = 1.0f / s;
+
+  if (vec) {
+#pragma unroll
+    for (int i = 0; i < EPT / 8; ++i) {
+      const int e = (tid + i * T) * 8;
+      if (e < N) {
+        uint4 w;
+        w.x = bf16x2_bits(x[i * 8 + 0] * inv, x[i * 8 + 1] * inv);
+        w.y = bf16x2_bits(x[i * 8 + 2] * inv, x[i * 8 + 3] * inv);
+        w.z = bf16x2_bits(x[i * 8 + 4] * inv, x[i * 8 + 5] * inv);
+        w.w = bf16x2_bits(x[i * 8 + 6] * inv, x[i * 8 + 7] * inv);
+        *reinterpret_cast<uint4*>(prow + e) = w;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      const int e = tid + i * T;
+      if (e < N) {
+        __nv_bfloat16 h = __float2bfloat16_rn(x[i] * inv);
+        prow[e] = *reinterpret_cast<uint16_t*>(&h);
+      }
+    }
+  }
+  if (tid == 0) lse[row] = m + logf(s);
+}
+
+// ----------------------------------------------------------------- values
+// O tile of 128 rows x D per CTA; 8 warps, each 16 rows x D; keys in chunks
+// of 64 with the next chunk prefetched into registers during the MMAs.
+template <int D>
+__global__ void __launch_bounds__(256) naive_values_kernel(const uint16_t* __restrict__ P,
+                                                           const uint16_t* __restrict__ V,
+                                                           uint16_t* __restrict__ O, int N) {
+  constexpr int LDP = kChunk + 8;
+  constexpr int LDV = D + 8;
+  constexpr int PV = kT * kChunk / 8 / 256;  // uint4 of P per thread per chunk (4)
+  constexpr int VV = kChunk * D / 8 / 256;   // uint4 of V per thread per chunk (2 or 4)
+  extern __shared__ __align__(16) uint16_t sm[];
+  uint16_t* Ps = sm;
+  uint16_t* Vs = sm + kT * LDP;
+  const int r0 = blockIdx.x * kT, bh = blockIdx.y;
+  const size_t head = static_cast<size_t>(bh) * N;
+  const uint16_t* Ph = P + head * N;
+  const uint16_t* Vh = V + head * D;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const bool vec_ok = (N % 8) == 0;
+
+  uint4 pr[PV], vr[VV];
+  auto fetch = [&](int kv0) {
+#pragma unroll
+    for (int i = 0; i < PV; ++i) {
+      const int e = tid + i * 256, r = e / (kChunk / 8), cv = (e % (kChunk / 8)) * 8;
+      const int valid = (r0 + r < N) ? max(0, min(8, N - (kv0 + cv))) : 0;
+      pr[i] = valid > 0 ? load8(Ph + static_cast<size_t>(r0 + r) * N + kv0 + cv, valid, vec_ok)
+                        : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < VV; ++i) {
+      const int e = tid + i * 256, r = e / (D / 8), cv = (e % (D / 8)) * 8;
+      vr[i] = (kv0 + r < N) ? *reinterpret_cast<const uint4*>(Vh + static_cast<size_t>(kv0 + r) * D + cv)
+                            : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto stash = [&]() {
+#pragma unroll
+    for (int i = 0; i < PV; ++i) {
+      const int e = tid + i * 256, r = e / (kChunk / 8), cv = (e % (kChunk / 8)) * 8;
+      *reinterpret_cast<uint4*>(Ps + r * LDP + cv) = pr[i];
+    }
+#pragma unroll
+    for (int i = 0; i < VV; ++i) {
+      const int e = tid + i * 256, r = e / (D / 8), cv = (e % (D / 8)) * 8;
+      *reinterpret_cast<uint4*>(Vs + r * LDV + cv) = vr[i];
+    }
+  };
+
+  float acc[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[n][u] = 0.0f;
+
+  fetch(0);
+  for (int kv0 = 0; kv0 < N; kv0 += kChunk) {
+    stash();
+    __syncthreads();
+    if (kv0 + kChunk < N) fetch(kv0 + kChunk);
+#pragma unroll
+    for (int kk = 0; kk < kChunk; kk += 16) {
+      uint32_t a[4];
+      ldsm_x4(smem_addr(Ps + (warp * 16 + (lane % 16)) * LDP + kk + (lane / 16) * 8), a);
+#pragma unroll
+      for (int nb = 0; nb < D / 16; ++nb) {
+        uint32_t b[4];
+        ldsm_x4_trans(smem_addr(Vs + (kk + (lane % 16)) * LDV + nb * 16 + (lane / 16) * 8), b);
+        mma16816(acc[2 * nb], a, b[0], b[1]);
+        mma16816(acc[2 * nb + 1], a, b[2], b[3]);
+      }
+    }
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = r0 + warp * 16 + lane / 4 + 8 * h;
+      const int c = n * 8 + (lane % 4) * 2;
+      if (r < N)
+        *reinterpret_cast<uint32_t*>(O + (head + r) * D + c) =
+            bf16x2_bits(acc[n][2 * h], acc[n][2 * h + 1]);
+    }
+}
+
+template <int D>
+int launch_naive_d(const AttnArgs& a, void* workspace, cudaStream_t stream) {
+  const int N = a.N, BH = a.B * a.H;
+  uint16_t* S = static_cast<uint16_t*>(workspace);
+  uint16_t* P = S + static_cast<size_t>(BH) * N * N;
+  const auto* q = static_cast<const uint16_t*>(a.q);
+  const auto* k = static_cast<const uint16_t*>(a.k);
+  const auto* v = static_cast<const uint16_t*>(a.v);
+  auto* o = static_cast<uint16_t*>(a.o);
+  const int tiles = (N + kT - 1) / kT;
+  if (BH > 65535) return ATTN_ERR_SHAPE;
+
+  const int smem_scores = 2 * kT * (D + 8) * 2;
+  if (cudaFuncSetAttribute(naive_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_scores) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  naive_scores_kernel<D><<<dim3(tiles, tiles, BH), 256, smem_scores, stream>>>(q, k, S, N, a.scale,
+                                                                              a.causal);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+
+  // softmax launch shape: EPT elements per thread, T threads per row
+  int ept = 8;
+  while (ept < 64 && (N + ept - 1) / ept > 256) ept *= 2;
+  int T = ((N + ept - 1) / ept + 31) / 32 * 32;
+  if (T > 512) return ATTN_ERR_SHAPE;
+  const unsigned rows = static_cast<unsigned>(static_cast<size_t>(BH) * N);
+  switch (ept) {
+    case 8: naive_softmax_kernel<8><<<rows, T, 0, stream>>>(S, P, a.lse, N); break;
+    case 16: naive_softmax_kernel<16><<<rows, T, 0, stream>>>(S, P, a.lse, N); break;
+    case 32: naive_softmax_kernel<32><<<rows, T, 0, stream>>>(S, P, a.lse, N); break;
+    default: naive_softmax_kernel<64><<<rows, T, 0, stream>>>(S, P, a.lse, N); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+
+  const int smem_values = (kT * (kChunk + 8) + kChunk * (D + 8)) * 2;
+  if (cudaFuncSetAttribute(naive_values_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_values) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  naive_values_kernel<D><<<dim3(tiles, BH), 256, smem_values, stream>>>(P, v, o, N);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+}  // namespace
+
+int launch_naive(const AttnArgs& a, void* workspace, cudaStream_t stream) {
+  return a.d == 128 ? launch_naive_d<128>(a, workspace, stream)
+                    : launch_naive_d<64>(a, workspace, stream);
+}
+
+}  // namespace attn

@@ -1,0 +1,139 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) exact-attention forward library
+ * (libattn_b200.so).
+ *
+ * The operation is exact scaled dot-product attention,
+ *
+ *     O = softmax(Q K^T * scale  [+ causal mask]) V,
+ *
+ * with the row-wise softmax and the three steps (scores, softmax, output) as
+ * described on the grasp.study lesson "The Computational Steps of Standard
+ * Self-Attention" and on the anylearn.cc page "Attention Is Memory-Bound, and
+ * Nobody Noticed for Five Years". attn_fwd computes it as one fused tiled
+ * kernel that never writes the N x N score or probability matrix to HBM
+ * (pratikdhanave.com, "The Attention Bottleneck - and How FlashAttention Fixed
+ * It", section "The fix: tiling and fusion, never touch HBM"); attn_fwd_naive
+ * computes the same function as three separate kernels that materialise S and
+ * P in HBM (the "standard path" of the anylearn.cc page).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers q, k, v, o, lse, workspace are DEVICE pointers owned by the
+ *   caller. The library never allocates or frees device memory, never
+ *   synchronises the stream, and keeps no per-call state, so calls on
+ *   different streams are independent.
+ * - q, k, v, o: bf16 (IEEE binary16-brain, 2 bytes), layout [B, H, N, d]
+ *   contiguous, i.e. element (b, h, i, c) at ((b*H + h)*N + i)*d + c. Must be
+ *   16-byte aligned.
+ * - lse: fp32 [B, H, N] contiguous, 4-byte aligned. lse[b,h,i] is the natural
+ *   logarithm of sum_j exp(scale * q_i . k_j) over the allowed keys j.
+ * - d (head dimension) must be 64 or 128 (the page's "d is 64 or 128").
+ * - B, H, N >= 1; B*H*N must fit in a signed 32-bit int.
+ * - scale: the logit multiplier (1/sqrt(d) for standard attention), applied
+ *   as given; must be finite and > 0.
+ * - causal: 0 (every key) or 1 (key j allowed for query i iff j <= i).
+ * - Arithmetic: bf16 operands, fp32 accumulation, fp32 softmax; O is rounded
+ *   to bf16 (round to nearest even).
+ * - Return value: ATTN_OK (0) or a negative ATTN_ERR_* code. On an argument
+ *   error nothing is launched. A kernel that launched fine but failed on the
+ *   device (the bounded-wait watchdog fired) is reported by
+ *   attn_last_device_error().
+ * - Asynchrony: work is enqueued on `stream` (a cudaStream_t; 0 = legacy
+ *   default stream) and completes in stream order; errors of the kernel
+ *   itself surface at the caller's next synchronisation.
+ * - Device: an sm_100 (B200-class) device must be current; otherwise
+ *   ATTN_ERR_UNSUPPORTED_DEVICE.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *attn_stream_t; /* same type as cudaStream_t */
+
+enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = -1,               /* a required pointer is NULL */
+    ATTN_ERR_SHAPE = -2,              /* B, H or N < 1, or B*H*N too large */
+    ATTN_ERR_HEADDIM = -3,            /* d is not 64 or 128 */
+    ATTN_ERR_ALIGN = -4,              /* a pointer breaks its alignment rule */
+    ATTN_ERR_SCALE = -5,              /* scale is not finite, or <= 0 */
+    ATTN_ERR_CAUSAL = -6,             /* causal is not 0 or 1 */
+    ATTN_ERR_WORKSPACE = -7,          /* naive path: workspace too small */
+    ATTN_ERR_LAUNCH = -8,             /* the CUDA launch failed */
+    ATTN_ERR_UNSUPPORTED_DEVICE = -9, /* current device is not sm_100 */
+    ATTN_ERR_TIMEOUT = -10,           /* a kernel gave up on a bounded wait */
+    ATTN_ERR_CUDA = -11               /* another CUDA runtime/driver call failed */
+};
+
+/*
+ * attn_fwd - fused exact attention forward (the hot path).
+ *
+ * One persistent-style grid of warp-specialised CTAs: TMA loads Q, K, V tiles
+ * into swizzled shared memory through an mbarrier ring, tcgen05 MMAs
+ * accumulate S = Q K^T and O += P V in tensor memory, and softmax warps keep a
+ * running row maximum and row sum (online softmax, exp2 domain). S and P never
+ * leave the SM; only O and lse are written.
+ *
+ * q, k, v (in), o (out): [B, H, N, d] bf16. lse (out): [B, H, N] fp32.
+ * Returns ATTN_OK or ATTN_ERR_*; see the conventions above.
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int H, int N, int d, float scale, int causal,
+             attn_stream_t stream);
+
+/*
+ * attn_fwd_naive_workspace_bytes - bytes of workspace attn_fwd_naive needs:
+ * 2 * (B*H*N*N) bf16 values (S, then P), i.e. 4*B*H*N*N bytes. Returns 0 if
+ * the arguments are not positive or the size overflows.
+ */
+size_t attn_fwd_naive_workspace_bytes(int B, int H, int N);
+
+/*
+ * attn_fwd_naive - the deliberately unfused standard path: three kernels on
+ * `stream`,
+ *   1. S = scale * Q K^T   (causally masked entries set to -inf), bf16, to HBM
+ *   2. P = softmax(S) row-wise, bf16, to HBM; lse in fp32
+ *   3. O = P V, bf16
+ * so each N x N matrix crosses the HBM boundary twice (four crossings in all,
+ * as the anylearn.cc page counts them). Same arguments and result as
+ * attn_fwd, plus a caller-owned device workspace of at least
+ * attn_fwd_naive_workspace_bytes(B, H, N) bytes, 16-byte aligned (S at offset
+ * 0, P right after it). Extra limits: N <= 32768 and B*H <= 65535
+ * (ATTN_ERR_SHAPE otherwise). A smaller workspace returns ATTN_ERR_WORKSPACE.
+ */
+int attn_fwd_naive(const void *q, const void *k, const void *v, void *o,
+                   float *lse, int B, int H, int N, int d, float scale,
+                   int causal, void *workspace, size_t workspace_bytes,
+                   attn_stream_t stream);
+
+/*
+ * attn_last_device_error - reads and clears the device-side error word of the
+ * current device. Every wait inside the fused kernel is bounded; a CTA whose
+ * wait runs out sets this word, drains its own copies, frees its tensor memory
+ * and exits. Returns ATTN_OK, ATTN_ERR_TIMEOUT, or ATTN_ERR_CUDA if the query
+ * itself failed. Synchronises `stream` (the only entry point that does).
+ */
+int attn_last_device_error(attn_stream_t stream);
+
+/* attn_status_string - a static, human-readable name for a status code. */
+const char *attn_status_string(int status);
+
+/*
+ * attn_selftest_wait_timeout - watchdog check. Launches one CTA that waits, with
+ * the same bounded wait the fused kernel uses, on an mbarrier nothing ever
+ * arrives on, with a limit of `limit_ms` milliseconds (1..5000). The kernel then
+ * records the timeout and returns; the device stays usable. After a stream
+ * synchronisation attn_last_device_error() must report ATTN_ERR_TIMEOUT.
+ */
+int attn_selftest_wait_timeout(int limit_ms, attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,69 @@
+"""Comparison helpers for the GPU parity tests.
+
+Tolerances are the ones the method is held to: on O, max-abs error <= 2e-2
+and mean-abs error <= 2e-3 over every checked element; on the log-sum-exp,
+|error| <= 1e-3 * max(1, |lse_ref|) (a relative bound that stays meaningful
+when lse is near 0, e.g. the first causal row where lse = s_00).
+"""
+import numpy as np
+import torch
+
+import oracle
+from exact_attention_125_b200.inputs import gather_rows, sample_rows
+
+O_MAX_ABS = 2e-2
+O_MEAN_ABS = 2e-3
+LSE_REL = 1e-3
+
+
+def compare(o_gpu_rows, lse_gpu_rows, o_ref, lse_ref):
+    """Returns a dict of error figures; o_* are [R, d], lse_* are [R]."""
+    o = o_gpu_rows.float().cpu().numpy().astype(np.float64)
+    lse = lse_gpu_rows.float().cpu().numpy().astype(np.float64)
+    err = np.abs(o - o_ref)
+    lse_err = np.abs(lse - lse_ref) / np.maximum(1.0, np.abs(lse_ref))
+    return {
+        "o_max_abs": float(err.max()) if err.size else 0.0,
+        "o_mean_abs": float(err.mean()) if err.size else 0.0,
+        "lse_max_rel": float(lse_err.max()) if lse_err.size else 0.0,
+        "finite": bool(np.isfinite(o).all() and np.isfinite(lse).all()),
+    }
+
+
+def assert_within(e, what=""):
+    assert e["finite"], f"{what}: non-finite output {e}"
+    assert e["o_max_abs"] <= O_MAX_ABS, f"{what}: O max-abs {e}"
+    assert e["o_mean_abs"] <= O_MEAN_ABS, f"{what}: O mean-abs {e}"
+    assert e["lse_max_rel"] <= LSE_REL, f"{what}: lse {e}"
+
+
+def check_against_oracle(q, k, v, o, lse, scale, causal, rows=None, what=""):
+    """q, k, v: CPU bf16 [B,H,N,d]; o, lse: GPU outputs. rows=None: all rows."""
+    B, H, N, d = q.shape
+    if rows is None:
+        rows = oracle.all_rows(B * H, N)
+    o_ref, lse_ref = oracle.attention(q, k, v, scale, causal, rows=rows)
+    o_rows = gather_rows(o.cpu(), rows)
+    lse_rows = gather_rows(lse.cpu().unsqueeze(-1), rows).squeeze(-1)
+    e = compare(o_rows, lse_rows, o_ref, lse_ref)
+    assert_within(e, what)
+    return e
+
+
+def sampled(w):
+    return sample_rows(w.seed, w.B * w.H, w.N, 256)
+
+
+def to_gpu(*ts):
+    return tuple(t.to("cuda") for t in ts)
+
+
+def scale_of(d):
+    return 1.0 / float(np.sqrt(d))
+
+
+def empty_outputs(q):
+    B, H, N, d = q.shape
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    return o, lse

@@ -1,0 +1,91 @@
+"""The C-ABI library: it loads, exports every function include/attn.h
+declares, and rejects bad arguments before any device work (no GPU needed)."""
+import os
+import re
+
+import pytest
+
+import exact_attention_125_b200 as ea
+from exact_attention_125_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return ea.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("attn_fwd", "attn_fwd_naive", "attn_fwd_naive_workspace_bytes",
+                 "attn_last_device_error", "attn_status_string"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in ea.STATUS.items():
+        assert ea.abi.attn_status_string(code).startswith(name)
+
+
+A = 0x100000  # a 16-byte aligned fake device address; never dereferenced
+
+
+def _fwd(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, scale=0.125, causal=0,
+                stream=None)
+    args.update(kw)
+    return ea.abi.attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"],
+                           args["H"], args["N"], args["d"], args["scale"], args["causal"],
+                           args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(lse=None), -1),
+    (dict(B=0), -2), (dict(N=0), -2), (dict(H=-3), -2), (dict(B=65536, H=65536), -2),
+    (dict(d=96), -3), (dict(d=256), -3),
+    (dict(q=A + 8), -4), (dict(o=A + 2), -4), (dict(lse=A + 2), -4),
+    (dict(scale=float("nan")), -5), (dict(scale=float("inf")), -5), (dict(scale=0.0), -5),
+    (dict(scale=-0.5), -5),
+    (dict(causal=2), -6),
+])
+def test_fused_argument_errors(L, kw, code):
+    assert _fwd(**kw) == code
+
+
+def test_naive_argument_errors(L):
+    n = ea.abi.attn_fwd_naive_workspace_bytes(1, 1, 128)
+    assert n == 4 * 128 * 128
+    assert ea.abi.attn_fwd_naive_workspace_bytes(8, 32, 8192) == 4 * 8 * 32 * 8192 * 8192
+    assert ea.abi.attn_fwd_naive_workspace_bytes(0, 1, 1) == 0
+    f = ea.abi.attn_fwd_naive
+    assert f(A, A, A, A, A, 1, 1, 128, 64, 0.1, 0, None, n, None) == -1
+    assert f(A, A, A, A, A, 1, 1, 128, 64, 0.1, 0, A + 4, n, None) == -4
+    assert f(A, A, A, A, A, 1, 1, 128, 64, 0.1, 0, A, n - 1, None) == -7
+    assert f(A, A, A, A, A, 1, 1, 40000, 64, 0.1, 0, A, 1 << 40, None) == -2
+
+
+def test_selftest_argument_range(L):
+    assert ea.abi.attn_selftest_wait_timeout(0, None) == -2
+    assert ea.abi.attn_selftest_wait_timeout(6000, None) == -2
+
+
+def test_product_path_has_no_fallback(monkeypatch):
+    # with the library missing, the binding raises instead of computing
+    monkeypatch.setattr(ea, "_lib", None)
+    monkeypatch.setattr(ea, "_LIB_PATH", "/nonexistent/libattn_b200.so")
+    with pytest.raises(RuntimeError):
+        ea.lib()

@@ -1,0 +1,123 @@
+"""attn_fwd (fused tcgen05 kernel) against the fp64 oracle, element by element.
+
+Small and ragged shapes compare every row; the large workloads compare a
+seeded sample of 256 query rows per (batch, head), rows 0 and N-1 included,
+in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_125_b200 as ea
+from exact_attention_125_b200.inputs import WORKLOADS, make_qkv, make_workload
+from parity_util import (check_against_oracle, empty_outputs, sampled, scale_of,
+                         to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    # B, H, N, d, causal
+    (1, 1, 128, 64, False),
+    (1, 1, 128, 128, True),
+    (1, 1, 1, 64, False),
+    (1, 1, 1, 128, True),
+    (1, 2, 2, 64, True),
+    (2, 1, 127, 64, True),
+    (1, 1, 129, 128, False),
+    (1, 2, 255, 128, True),
+    (1, 1, 257, 64, False),
+    (1, 1, 1000, 128, True),
+    (2, 3, 384, 128, False),
+    (1, 2, 640, 64, True),
+    (1, 1, 1000, 64, False),
+]
+
+
+def _run(q, k, v, scale, causal):
+    qg, kg, vg = to_gpu(q, k, v)
+    o, lse = empty_outputs(qg)
+    ea.attn_fwd(qg, kg, vg, o, lse, scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    assert ea.last_device_error() == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", SMALL)
+def test_small_shapes_all_rows(B, H, N, d, causal):
+    q, k, v = make_qkv(B, H, N, d, seed=N * 7 + d + int(causal))
+    o, lse = _run(q, k, v, scale_of(d), causal)
+    check_against_oracle(q, k, v, o, lse, scale_of(d), causal, what=f"{(B, H, N, d, causal)}")
+
+
+@pytest.mark.parametrize("name", ["single_head_128", "bert_base_1024"])
+def test_workloads_all_rows(name):
+    w = WORKLOADS[name]
+    q, k, v = make_workload(w)
+    o, lse = _run(q, k, v, w.scale, w.causal)
+    check_against_oracle(q, k, v, o, lse, w.scale, w.causal, what=name)
+
+
+@pytest.mark.parametrize("name", ["decoder_2048_causal", "long_8192_causal",
+                                  "stress_65536_causal"])
+def test_workloads_sampled_rows(name):
+    w = WORKLOADS[name]
+    q, k, v = make_workload(w)
+    o, lse = _run(q, k, v, w.scale, w.causal)
+    e = check_against_oracle(q, k, v, o, lse, w.scale, w.causal, rows=sampled(w), what=name)
+    print(name, e)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_constant_values(d, causal):
+    # V rows all equal to c: every O row is c (probability rows sum to 1).
+    B, H, N = 1, 2, 300
+    q, k, _ = make_qkv(B, H, N, d, seed=5)
+    c = torch.linspace(-2, 2, d).to(torch.bfloat16)
+    v = c.expand(B, H, N, d).contiguous()
+    o, _ = _run(q, k, v, scale_of(d), causal)
+    err = (o.float().cpu() - c.float()).abs().max().item()
+    assert err <= 2e-2
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_single_key_and_causal_first_row(d):
+    q, k, v = make_qkv(1, 3, 1, d, seed=11)
+    o, lse = _run(q, k, v, scale_of(d), False)
+    assert torch.equal(o.cpu(), v)  # exactly v0: p = 1, bf16 round trip exact
+    want = (q.double() * k.double()).sum(-1) * scale_of(d)
+    assert (lse.cpu().double() - want).abs().max().item() <= 1e-3 * max(1.0, want.abs().max().item())
+    q, k, v = make_qkv(2, 2, 333, d, seed=12)
+    o, _ = _run(q, k, v, scale_of(d), True)
+    assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_per_row_logit_shift(causal):
+    # K' = K + 1 u^T with entries on the 1/8 grid (exact in bf16): O is
+    # unchanged and lse moves by scale * q_i . u (exact in the oracle).
+    B, H, N, d = 1, 2, 260, 128
+    q, k, v = make_qkv(B, H, N, d, seed=21, dist="grid8")
+    u = make_qkv(1, 1, 1, d, seed=22, dist="grid8")[0].reshape(d)
+    k2 = (k.float() + u.float()).to(torch.bfloat16)
+    assert torch.equal(k2.float(), k.float() + u.float())
+    scale = scale_of(d)
+    o1, l1 = _run(q, k, v, scale, causal)
+    o2, l2 = _run(q, k2, v, scale, causal)
+    shift = (q.double() @ u.double()) * scale
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+    dl = (l2.cpu().double() - l1.cpu().double() - shift).abs()
+    assert dl.max().item() <= 1e-3 * max(1.0, l1.abs().max().item())
+
+
+def test_outputs_do_not_depend_on_stale_memory():
+    # outputs are fully overwritten: prefill with NaN, compare two runs
+    q, k, v = make_qkv(1, 2, 200, 64, seed=3)
+    qg, kg, vg = to_gpu(q, k, v)
+    o = torch.full((1, 2, 200, 64), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((1, 2, 200), float("nan"), dtype=torch.float32, device="cuda")
+    ea.attn_fwd(qg, kg, vg, o, lse, causal=True)
+    o2, l2 = ea.attn_fwd(qg, kg, vg, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
