@@ -5,7 +5,7 @@ import torch
 
 import exact_attention_125_b200 as ea
 from exact_attention_125_b200.inputs import WORKLOADS, make_qkv, make_workload
-from parity_util import (check_against_oracle, empty_outputs, sampled, scale_of,
+from parity_util import (check_naive_against_oracle, empty_outputs, sampled, scale_of,
                          to_gpu)
 
 pytestmark = pytest.mark.gpu
@@ -32,21 +32,22 @@ def _run(q, k, v, scale, causal):
 def test_small_shapes(B, H, N, d, causal):
     q, k, v = make_qkv(B, H, N, d, seed=N + d)
     o, lse = _run(q, k, v, scale_of(d), causal)
-    check_against_oracle(q, k, v, o, lse, scale_of(d), causal, what=f"naive {(B, H, N, d)}")
+    check_naive_against_oracle(q, k, v, o, lse, scale_of(d), causal, what=f"naive {(B, H, N, d)}")
 
 
 def test_bert_base_all_rows():
     w = WORKLOADS["bert_base_1024"]
     q, k, v = make_workload(w)
     o, lse = _run(q, k, v, w.scale, w.causal)
-    check_against_oracle(q, k, v, o, lse, w.scale, w.causal, what="naive bert")
+    check_naive_against_oracle(q, k, v, o, lse, w.scale, w.causal, what="naive bert")
 
 
 def test_decoder_sampled():
     w = WORKLOADS["decoder_2048_causal"]
     q, k, v = make_workload(w)
     o, lse = _run(q, k, v, w.scale, w.causal)
-    check_against_oracle(q, k, v, o, lse, w.scale, w.causal, rows=sampled(w), what="naive dec")
+    check_naive_against_oracle(q, k, v, o, lse, w.scale, w.causal, rows=sampled(w),
+                               what="naive dec")
 
 
 def test_naive_and_fused_agree():
