@@ -18,7 +18,12 @@ import threading
 __all__ = [
     "AttnError", "lib", "attn_fwd", "attn_fwd_naive", "naive_workspace_bytes",
     "last_device_error", "status_string", "selftest_wait_timeout", "abi",
+    "NOALLOC_SCRATCH_BYTES",
 ]
+
+# Size of the library-owned scratch array behind attn_fwd_naive_noalloc
+# (ATTN_NOALLOC_SCRATCH_BYTES in include/attn.h).
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_b200.so")
 _lock = threading.Lock()
@@ -57,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_naive_workspace_bytes.restype = sz
         L.attn_fwd_naive.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
         L.attn_fwd_naive.restype = i
+        L.attn_fwd_naive_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.attn_fwd_naive_noalloc.restype = i
         L.attn_last_device_error.argtypes = [vp]
         L.attn_last_device_error.restype = i
         L.attn_status_string.argtypes = [i]
@@ -82,6 +89,10 @@ class abi:
     @staticmethod
     def attn_fwd_naive_workspace_bytes(B, H, N) -> int:
         return int(lib().attn_fwd_naive_workspace_bytes(B, H, N))
+
+    @staticmethod
+    def attn_fwd_naive_noalloc(q, k, v, o, lse, B, H, N, d, scale, causal, stream) -> int:
+        return lib().attn_fwd_naive_noalloc(q, k, v, o, lse, B, H, N, d, scale, causal, stream)
 
     @staticmethod
     def attn_last_device_error(stream) -> int:

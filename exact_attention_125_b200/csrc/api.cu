@@ -101,6 +101,22 @@ int attn_fwd_naive(const void* q, const void* k, const void* v, void* o, float* 
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
+int attn_fwd_naive_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int H, int N, int d, float scale, int causal,
+                           attn_stream_t stream) {
+  int st = validate(q, k, v, o, lse, B, H, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (N > 32768 || static_cast<long long>(B) * H > 65535) return ATTN_ERR_SHAPE;
+  const size_t need = attn_fwd_naive_workspace_bytes(B, H, N);
+  if (need == 0 || need > static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES))
+    return ATTN_ERR_WORKSPACE;
+  if ((st = check_device()) != ATTN_OK) return st;
+  void* scratch = attn::noalloc_scratch_ptr();
+  if (!scratch) return ATTN_ERR_CUDA;
+  return attn::launch_naive(pack(q, k, v, o, lse, B, H, N, d, scale, causal), scratch,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
 int attn_last_device_error(attn_stream_t stream) {
   return attn::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream));
 }

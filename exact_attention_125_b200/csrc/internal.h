@@ -25,6 +25,10 @@ int launch_fused(const AttnArgs& a, cudaStream_t stream);
 // Unfused three-kernel path (naive.cu). Arguments already validated.
 int launch_naive(const AttnArgs& a, void* workspace, cudaStream_t stream);
 
+// Device address of the fixed scratch array used by attn_fwd_naive_noalloc on
+// the current device (naive.cu); nullptr if the lookup failed.
+void* noalloc_scratch_ptr();
+
 // Device error word of the current device (fused_fwd.cu).
 int read_and_clear_device_error(cudaStream_t stream);
 

@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/attn.h"
 #include "internal.h"
@@ -393,6 +394,29 @@ int launch_naive_d(const AttnArgs& a, void* workspace, cudaStream_t stream) {
 int launch_naive(const AttnArgs& a, void* workspace, cudaStream_t stream) {
   return a.d == 128 ? launch_naive_d<128>(a, workspace, stream)
                     : launch_naive_d<64>(a, workspace, stream);
+}
+
+// ------------------------------------------------- no-allocation variant
+// Scratch for attn_fwd_naive_noalloc: S and P live here instead of in a
+// caller-provided workspace. The array is part of the library image, so every
+// GPU that loads the library reserves it until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress once per device (with that device current) and cached.
+void* noalloc_scratch_ptr() {
+  static void* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
 }
 
 }  // namespace attn

@@ -112,6 +112,41 @@ int attn_fwd_naive(const void *q, const void *k, const void *v, void *o,
                    attn_stream_t stream);
 
 /*
+ * ATTN_NOALLOC_SCRATCH_BYTES - size of the fixed device scratch array behind
+ * attn_fwd_naive_noalloc (64 MiB). Every GPU that loads the library holds it
+ * until the process exits.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * attn_fwd_naive_noalloc - attn_fwd_naive for callers that must not allocate
+ * device memory. The pages describe no such entry point: it has no
+ * counterpart there. It exists for callers that cannot call cudaMalloc or
+ * hand over a workspace: code embedded in a host framework that owns the
+ * whole device-memory budget through its own pool and forbids allocations
+ * outside it, and latency-bound loops where cudaMalloc/cudaFree would add
+ * their implicit device-wide synchronisation.
+ *
+ * Same arguments, limits and result as attn_fwd_naive, minus the workspace:
+ * S and P go to a library-owned device array of ATTN_NOALLOC_SCRATCH_BYTES,
+ * so 4*B*H*N*N must not exceed it (ATTN_ERR_WORKSPACE otherwise, before any
+ * launch). The function allocates nothing itself: no cudaMalloc, cudaFree or
+ * allocating library call.
+ *
+ * - Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture on that device.
+ * - Sharing: every call on a device uses the same array, which keeps the
+ *   previous call's contents. The three kernels overwrite every element of S
+ *   and P they read, so nothing has to start at zero. Calls whose work
+ *   overlaps on the GPU (different streams without ordering between them)
+ *   race on the array and give wrong results; order them on one stream.
+ */
+int attn_fwd_naive_noalloc(const void *q, const void *k, const void *v,
+                           void *o, float *lse, int B, int H, int N, int d,
+                           float scale, int causal, attn_stream_t stream);
+
+/*
  * attn_last_device_error - reads and clears the device-side error word of the
  * current device. Every wait inside the fused kernel is bounded; a CTA whose
  * wait runs out sets this word, drains its own copies, frees its tensor memory
