@@ -55,12 +55,31 @@ namespace {
 
 constexpr int kTileRows = 128;           // query rows per tile == keys per KV tile
 constexpr int kBlockRows = 256;          // query rows per CTA (two tiles)
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // three warpgroups
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;     // warps 10 and 11 only give their registers away
+// Registers per thread: what ptxas allocates at launch for 384 threads (the
+// host refuses to launch otherwise), and the split after setmaxnreg. The
+// split uses exactly the launch total.
+constexpr int kRegsAtLaunch = 168;
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsOther = 56;
+static_assert(128 * (2 * kRegsSoftmax + kRegsOther) == kThreads * kRegsAtLaunch,
+              "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 256 while m lags
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// K/V tiles the producer asks L2 to fetch ahead of the ones already in the
+// shared-memory ring (0 = no prefetch).
+constexpr int kPrefetchTiles = 0;
+
+// Which of a row's 64 (even, odd) column pairs take the FMA-pipe exponential
+// (exp2_poly_pair) instead of the MUFU one; kPolyPeriod = 0 means none.
+constexpr int kPolyPeriod = 4;
+__host__ __device__ constexpr bool poly_pair(int cc) {
+  return kPolyPeriod > 0 && cc % (kPolyPeriod > 0 ? kPolyPeriod : 1) == kPolyPeriod - 1;
+}
 
 template <int D>
 struct Cfg {
@@ -129,9 +148,10 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
 #pragma unroll
     for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(sr[u]);
 #pragma unroll
-    for (int cc = 8; cc < 128; ++cc) mx[cc % 8] = fmaxf(mx[cc % 8], __uint_as_float(sr[cc]));
-    const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    for (int cc = 8; cc < 128; cc += 2)
+      mx[(cc / 2) % 8] = fmax3(mx[(cc / 2) % 8], __uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1]));
+    const float rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                             fmaxf(mx[6], mx[7]));
     const float m_tile = rmax * c;
     const bool raise = m_tile > m_run + kRescaleThreshold;
     const float m_new = raise ? m_tile : m_run;
@@ -151,19 +171,32 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     m_run = m_new;
     const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
 
-    float sum[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) sum[u] = 0.0f;
+    // p = 2^(s * c - m) for the 64 (even, odd) column pairs: scaling and
+    // summing in packed f32x2 form; most exponentials on the MUFU (ex2), the
+    // pairs poly_pair picks on the FMA pipe (exp2_poly_pair).
+    const uint64_t c2 = f2_pack(c, c);
+    const uint64_t nm2 = f2_pack(neg_m, neg_m);
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
     uint32_t pk[64];
 #pragma unroll
     for (int cc = 0; cc < 64; ++cc) {
-      const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * cc]), c, neg_m));
-      const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * cc + 1]), c, neg_m));
-      sum[(2 * cc) % 8] += p0;
-      sum[(2 * cc + 1) % 8] += p1;
+      float x0, x1, p0, p1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1])), c2, nm2),
+                x0, x1);
+      if (poly_pair(cc)) {
+        exp2_poly_pair(x0, x1, p0, p1);
+      } else {
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      acc[cc % 4] = f2_add(acc[cc % 4], f2_pack(p0, p1));
       pk[cc] = pack_bf16x2(p0, p1);
     }
-    l_run += ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+    {
+      float lo, hi;
+      f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
+      l_run += lo + hi;
+    }
     tmem_st_x64(tS, pk);
     tmem_st_wait();
     tc_fence_before_sync();
@@ -218,6 +251,15 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
                        q0 + g * kTileRows, bh, pol_q);
 
   const int n_loads = 2 * n_kv_b;  // K_0, V_0, K_1, V_1, ...
+  // L2 prefetch of the tiles kPrefetchTiles loads ahead of the ring.
+  auto prefetch = [&](int u) {
+    if (kPrefetchTiles > 0 && u < n_loads) {
+      const CUtensorMap* m = (u & 1) ? tv : tk;
+#pragma unroll
+      for (int a = 0; a < C::kAtoms; ++a) tma_prefetch_l2_3d(m, a * 64, (u >> 1) * kTileRows, bh);
+    }
+  };
+  for (int u = 0; u < kPrefetchTiles; ++u) prefetch(C::kStages + u);
   int t = 0;
   for (; t < n_loads; ++t) {
     const int slot = t % C::kStages;
@@ -232,6 +274,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
     for (int a = 0; a < C::kAtoms; ++a)
       tma_load_3d_hint(sRing + slot * C::kTileBytes + a * C::kAtomBytes, m, bar_full, a * 64,
                        j * kTileRows, bh, pol_kv);
+    prefetch(t + C::kStages + kPrefetchTiles);
   }
   // Teardown: every copy this thread issued must have landed before exit.
   drain_wait(bar_q, 0, wd);
@@ -384,12 +427,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Watchdog wd{abort_flag, p.err, p.wait_limit_ns};
 
   if (warp < 8) {
+    regs_increase<kRegsSoftmax>();
     const int g = warp / 4;
     softmax_role<D>(p, tmem, bars, bh, q0, g == 0 ? na : nb, g, wd);
-  } else if (warp == kProducerWarp) {
-    if (lane == 0) producer_role<D>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) mma_role<D>(tmem, base, bars, na, nb, wd);
+  } else {
+    regs_decrease<kRegsOther>();
+    if (warp == kProducerWarp) {
+      if (lane == 0) producer_role<D>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
+    } else if (warp == kMmaWarp) {
+      if (lane == 0) mma_role<D>(tmem, base, bars, na, nb, wd);
+    }
   }
   __syncwarp();
   tc_fence_before_sync();
@@ -488,6 +535,10 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream) {
   if (cudaFuncSetAttribute(fused_attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes) != cudaSuccess)
     return ATTN_ERR_CUDA;
+  // The register split inside the kernel assumes this exact allocation.
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, fused_attn_fwd_kernel<D>) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (fa.numRegs != kRegsAtLaunch || fa.maxThreadsPerBlock < kThreads) return ATTN_ERR_LAUNCH;
   fused_attn_fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
       mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
