@@ -36,7 +36,10 @@ if ROOT not in sys.path:
 WORKLOAD = "long_8192_causal"
 METRIC = "attn fwd TFLOP/s (causal-adjusted) and % of B200 dense BF16 peak"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_attn_fwd_long_8192_causal.txt")
-KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_125_b200", "csrc", "fused_fwd.cu")
+# the sources that define the fused kernel; the ncu summary records their hash
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_125_b200", "csrc", f)
+                  for f in ("fused_fwd.cu", "sm100.cuh", "tmem_io.cuh", "watchdog.cuh",
+                            "exp2_poly.cuh")]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -64,9 +67,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash(path=KERNEL_SOURCE) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_hash(paths=None) -> str:
+    h = hashlib.sha256()
+    for path in (paths or KERNEL_SOURCES):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic():

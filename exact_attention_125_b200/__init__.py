@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_selftest_wait_timeout.argtypes = [i, vp]
         L.attn_selftest_wait_timeout.restype = i
+        L.attn_selftest_exp2.argtypes = [vp, vp, i, vp]
+        L.attn_selftest_exp2.restype = i
         _lib = L
         return L
 
@@ -105,6 +107,10 @@ class abi:
     @staticmethod
     def attn_selftest_wait_timeout(limit_ms, stream) -> int:
         return lib().attn_selftest_wait_timeout(limit_ms, stream)
+
+    @staticmethod
+    def attn_selftest_exp2(x, y, n, stream) -> int:
+        return lib().attn_selftest_exp2(x, y, n, stream)
 
 
 def status_string(status: int) -> str:

@@ -128,6 +128,15 @@ int attn_selftest_wait_timeout(int limit_ms, attn_stream_t stream) {
   return attn::launch_wait_timeout_selftest(limit_ms, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int attn_selftest_exp2(const float* x, float* y, int n, attn_stream_t stream) {
+  if (!x || !y) return ATTN_ERR_NULL;
+  if (n < 1) return ATTN_ERR_SHAPE;
+  if (!aligned(x, 4) || !aligned(y, 4)) return ATTN_ERR_ALIGN;
+  int st = check_device();
+  if (st != ATTN_OK) return st;
+  return attn::launch_exp2_poly_selftest(x, y, n, reinterpret_cast<cudaStream_t>(stream));
+}
+
 const char* attn_status_string(int status) {
   switch (status) {
     case ATTN_OK: return "ATTN_OK";

@@ -32,6 +32,9 @@ void* noalloc_scratch_ptr();
 // Device error word of the current device (fused_fwd.cu).
 int read_and_clear_device_error(cudaStream_t stream);
 
+// exp2_poly self-test kernel (selftest.cu).
+int launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t stream);
+
 // Watchdog self-test kernel (fused_fwd.cu).
 int launch_wait_timeout_selftest(int limit_ms, cudaStream_t stream);
 

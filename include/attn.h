@@ -167,6 +167,16 @@ const char *attn_status_string(int status);
  */
 int attn_selftest_wait_timeout(int limit_ms, attn_stream_t stream);
 
+/*
+ * attn_selftest_exp2 - numerics check of the exponential the fused kernel
+ * evaluates on the FMA pipe for part of each softmax row (the rest uses the
+ * MUFU's ex2): 2^x by Cody-Waite range reduction (x = j + f, |f| <= 1/2) and a
+ * minimax cubic for 2^f, with j added to the exponent field; inputs below -125
+ * give a tiny positive value (<= 2^-124) in place of 0. x, y: n device floats,
+ * 4-byte aligned; y[i] = 2^x[i]. Launches one kernel on `stream`.
+ */
+int attn_selftest_exp2(const float *x, float *y, int n, attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
