@@ -70,10 +70,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 256 while m lags
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// K/V tiles the producer asks L2 to fetch ahead of the ones already in the
-// shared-memory ring (0 = no prefetch).
-constexpr int kPrefetchTiles = 0;
-
 // Which of a row's 64 (even, odd) column pairs take the FMA-pipe exponential
 // (exp2_poly_pair) instead of the MUFU one; kPolyPeriod = 0 means none.
 constexpr int kPolyPeriod = 4;
@@ -86,7 +82,8 @@ struct Cfg {
   static constexpr int kTileBytes = kTileRows * D * 2;  // one 128 x D bf16 tile
   static constexpr int kAtoms = D / 64;                 // 128-byte swizzle atoms per row
   static constexpr int kAtomBytes = kTileRows * 128;    // 16 KiB
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kStages = (D == 128) ? 4 : 8;  // tile slots of the ring
+  static constexpr int kUnits = kStages / 2;           // (V, K) units in flight
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
@@ -250,36 +247,38 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
       tma_load_3d_hint(sQ + g * C::kTileBytes + a * C::kAtomBytes, tq, bar_q, a * 64,
                        q0 + g * kTileRows, bh, pol_q);
 
-  const int n_loads = 2 * n_kv_b;  // K_0, V_0, K_1, V_1, ...
-  // L2 prefetch of the tiles kPrefetchTiles loads ahead of the ring.
-  auto prefetch = [&](int u) {
-    if (kPrefetchTiles > 0 && u < n_loads) {
-      const CUtensorMap* m = (u & 1) ? tv : tk;
-#pragma unroll
-      for (int a = 0; a < C::kAtoms; ++a) tma_prefetch_l2_3d(m, a * 64, (u >> 1) * kTileRows, bh);
-    }
-  };
-  for (int u = 0; u < kPrefetchTiles; ++u) prefetch(C::kStages + u);
-  int t = 0;
-  for (; t < n_loads; ++t) {
-    const int slot = t % C::kStages;
-    const uint32_t ph = (t / C::kStages) & 1;
-    const uint32_t bar_full = bars + 8u * (1 + slot);
-    const uint32_t bar_empty = bars + 8u * (1 + C::kStages + slot);
+  // K/V arrive in units that the MMA warp consumes together: unit 0 = K_0,
+  // unit u >= 1 = (V_{u-1}, K_u), the last unit V only. A unit occupies two
+  // tile slots of the ring (V in the first, K in the second) and has one full
+  // and one empty barrier, so the MMA warp waits once per step for its tiles.
+  const int n_units = n_kv_b + 1;
+  int u = 0;
+  for (; u < n_units; ++u) {
+    const int us = u % C::kUnits;
+    const uint32_t ph = (u / C::kUnits) & 1;
+    const uint32_t bar_full = bars + 8u * (1 + us);
+    const uint32_t bar_empty = bars + 8u * (1 + C::kStages + us);
     if (!wait_one(bar_empty, ph ^ 1u, wd)) break;
-    const CUtensorMap* m = (t & 1) ? tv : tk;
-    const int j = t >> 1;
-    mbar_arrive_expect_tx(bar_full, C::kTileBytes);
+    const bool has_v = u >= 1;
+    const bool has_k = u < n_kv_b;
+    mbar_arrive_expect_tx(bar_full, (int(has_v) + int(has_k)) * C::kTileBytes);
+    if (has_v) {
 #pragma unroll
-    for (int a = 0; a < C::kAtoms; ++a)
-      tma_load_3d_hint(sRing + slot * C::kTileBytes + a * C::kAtomBytes, m, bar_full, a * 64,
-                       j * kTileRows, bh, pol_kv);
-    prefetch(t + C::kStages + kPrefetchTiles);
+      for (int a = 0; a < C::kAtoms; ++a)
+        tma_load_3d_hint(sRing + (2 * us) * C::kTileBytes + a * C::kAtomBytes, tv, bar_full,
+                         a * 64, (u - 1) * kTileRows, bh, pol_kv);
+    }
+    if (has_k) {
+#pragma unroll
+      for (int a = 0; a < C::kAtoms; ++a)
+        tma_load_3d_hint(sRing + (2 * us + 1) * C::kTileBytes + a * C::kAtomBytes, tk, bar_full,
+                         a * 64, u * kTileRows, bh, pol_kv);
+    }
   }
   // Teardown: every copy this thread issued must have landed before exit.
   drain_wait(bar_q, 0, wd);
-  for (int u = (t > C::kStages ? t - C::kStages : 0); u < t; ++u)
-    drain_wait(bars + 8u * (1 + u % C::kStages), (u / C::kStages) & 1, wd);
+  for (int w = (u > C::kUnits ? u - C::kUnits : 0); w < u; ++w)
+    drain_wait(bars + 8u * (1 + w % C::kUnits), (w / C::kUnits) & 1, wd);
 }
 
 template <int D>
@@ -296,15 +295,17 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
 
-  auto slot_of = [](int t) { return t % C::kStages; };
-  auto par_of = [](int t) { return static_cast<uint32_t>((t / C::kStages) & 1); };
-  auto full_bar = [&](int t) { return bars + 8u * (1 + slot_of(t)); };
-  auto empty_bar = [&](int t) { return bars + 8u * (1 + C::kStages + slot_of(t)); };
+  // unit u (see producer_role): V_{u-1} in tile slot 2 (u % kUnits), K_u in the next one
+  auto par_of = [](int u) { return static_cast<uint32_t>((u / C::kUnits) & 1); };
+  auto full_bar = [&](int u) { return bars + 8u * (1 + u % C::kUnits); };
+  auto empty_bar = [&](int u) { return bars + 8u * (1 + C::kStages + u % C::kUnits); };
+  auto v_slot = [](int u) { return 2 * (u % C::kUnits); };
+  auto k_slot = [](int u) { return 2 * (u % C::kUnits) + 1; };
 
   // S_g = Q_g K^T : A = Q tile (K-major), B = K tile (K-major), 16-deep steps.
-  auto issue_qk = [&](int g, int t) {
+  auto issue_qk = [&](int g, int slot) {
     const uint32_t a0 = sQ + g * C::kTileBytes;
-    const uint32_t b0 = sRing + slot_of(t) * C::kTileBytes;
+    const uint32_t b0 = sRing + slot * C::kTileBytes;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t off = (kk >> 2) * C::kAtomBytes + (kk & 3) * 32;
@@ -313,8 +314,8 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
     }
   };
   // O_g += P_g V : A = P in tensor memory, B = V tile (MN-major), 16 keys per step.
-  auto issue_pv = [&](int g, int t, bool accumulate) {
-    const uint32_t b0 = sRing + slot_of(t) * C::kTileBytes;
+  auto issue_pv = [&](int g, int slot, bool accumulate) {
+    const uint32_t b0 = sRing + slot * C::kTileBytes;
 #pragma unroll
     for (int kk = 0; kk < kTileRows / 16; ++kk)
       mma_ts(tmem + C::col_o(g), tmem + C::col_s(g) + kk * 8,
@@ -325,24 +326,21 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   bool ok = wait_one(bar_q, 0, wd) && wait_one(full_bar(0), par_of(0), wd);
   if (ok) {
     tc_fence_after_sync();
-    issue_qk(0, 0);
+    issue_qk(0, k_slot(0));
     mma_commit(bar_s_full0);
-    issue_qk(1, 0);
+    issue_qk(1, k_slot(0));
     mma_commit(bar_s_full0 + 8u);
     mma_commit(empty_bar(0));
   }
   for (int j = 0; ok && j < nb; ++j) {
-    const int tv = 2 * j + 1;
-    const int tk = 2 * j + 2;
-    if (!(ok = wait_one(full_bar(tv), par_of(tv), wd))) break;
+    const int u = j + 1;  // V_j and K_{j+1}
+    if (!(ok = wait_one(full_bar(u), par_of(u), wd))) break;
     if (j < na) {
       if (!(ok = wait_one(bar_p_ready0, j & 1, wd))) break;
       tc_fence_after_sync();
-      issue_pv(0, tv, j > 0);
+      issue_pv(0, v_slot(u), j > 0);
       if (j + 1 < na) {
-        if (!(ok = wait_one(full_bar(tk), par_of(tk), wd))) break;
-        tc_fence_after_sync();
-        issue_qk(0, tk);
+        issue_qk(0, k_slot(u));
         mma_commit(bar_s_full0);
       } else {
         mma_commit(bar_o_final0);
@@ -350,17 +348,14 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
     }
     if (!(ok = wait_one(bar_p_ready0 + 8u, j & 1, wd))) break;
     tc_fence_after_sync();
-    issue_pv(1, tv, j > 0);
-    mma_commit(empty_bar(tv));
+    issue_pv(1, v_slot(u), j > 0);
     if (j + 1 < nb) {
-      if (!(ok = wait_one(full_bar(tk), par_of(tk), wd))) break;
-      tc_fence_after_sync();
-      issue_qk(1, tk);
+      issue_qk(1, k_slot(u));
       mma_commit(bar_s_full0 + 8u);
-      mma_commit(empty_bar(tk));
     } else {
       mma_commit(bar_o_final0 + 8u);
     }
+    mma_commit(empty_bar(u));
   }
   // Teardown: all MMAs this thread issued must be complete before the tensor
   // memory is freed.
