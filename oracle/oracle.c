@@ -23,6 +23,11 @@
  * -inf before the softmax means. A causal row always has key j = i, so no row
  * is empty; if a row were empty anyway the oracle writes o = 0, lse = -inf.
  *
+ * With fewer queries than keys (Nq <= Nk, the shape of generating new tokens
+ * against a long context) the Nq queries are the last Nq positions of the
+ * sequence: causally, query i may see keys j <= i + (Nk - Nq); for Nq = Nk
+ * that is the rule above.
+ *
  * The anylearn.cc page ("FlashAttention computes exactly the same function as
  * standard attention ... to within floating point reassociation") is why the
  * plain definition is the oracle for the fused kernel.
@@ -89,12 +94,10 @@ static void output_row(const double *p, const double *V, int n, int d, double *o
         for (int c = 0; c < d; ++c) o[c] += p[j] * V[(int64_t)j * d + c];
 }
 
-/* One query row of one head: steps 1-3 and the log-sum-exp. */
-static void attend_row(const double *q, const double *K, const double *V, int N,
-                       int d, double scale, int causal, int i, double *s_buf,
-                       double *o, double *lse) {
-    int nkeys = causal ? i + 1 : N;
-    if (nkeys > N) nkeys = N;
+/* One query row of one head: steps 1-3 and the log-sum-exp. nkeys is the
+ * number of allowed keys (a prefix of the head's keys). */
+static void attend_row(const double *q, const double *K, const double *V, int nkeys,
+                       int d, double scale, double *s_buf, double *o, double *lse) {
     if (nkeys <= 0) {
         for (int c = 0; c < d; ++c) o[c] = 0.0;
         *lse = -INFINITY;
@@ -107,6 +110,15 @@ static void attend_row(const double *q, const double *K, const double *V, int N,
     *lse = m + log(l);
 }
 
+/* Allowed keys of query i: all Nk, or those j <= i + (Nk - Nq) when causal. */
+static int allowed_keys(int i, int Nq, int Nk, int causal) {
+    if (!causal) return Nk;
+    long long n = (long long)i + (Nk - Nq) + 1;
+    if (n > Nk) n = Nk;
+    if (n < 0) n = 0;
+    return (int)n;
+}
+
 typedef struct {
     const void *q;
     int kind;
@@ -117,6 +129,7 @@ typedef struct {
     const int64_t *rows;  /* all (bh, i) pairs */
     const int64_t *mine;  /* indices into rows[] for this head */
     int64_t nmine;
+    int Nq;               /* query rows per head (N is the key count) */
     int tid, nthreads;
     double *o, *lse;
     int ok;        /* set to 1 by run_job when its rows are done */
@@ -136,10 +149,10 @@ static void *run_job(void *arg) {
     for (int64_t t = jb->tid; t < jb->nmine; t += jb->nthreads) {
         int64_t r = jb->mine[t];
         int i = (int)jb->rows[2 * r + 1];
-        int64_t qoff = (jb->bh * jb->N + i) * (int64_t)jb->d;
+        int64_t qoff = (jb->bh * jb->Nq + i) * (int64_t)jb->d;
         for (int c = 0; c < jb->d; ++c) qrow[c] = load_elem(jb->q, jb->kind, qoff + c);
-        attend_row(qrow, jb->K, jb->V, jb->N, jb->d, jb->scale, jb->causal, i, s,
-                   jb->o + r * (int64_t)jb->d, jb->lse + r);
+        attend_row(qrow, jb->K, jb->V, allowed_keys(i, jb->Nq, jb->N, jb->causal), jb->d,
+                   jb->scale, s, jb->o + r * (int64_t)jb->d, jb->lse + r);
     }
     free(s);
     free(qrow);
@@ -153,17 +166,18 @@ int oracle_default_threads(void) {
 }
 
 static int attend(const void *q, const void *k, const void *v, int kind, int B,
-                  int H, int N, int d, double scale, int causal,
+                  int H, int Nq, int N, int d, double scale, int causal,
                   const int64_t *rows, int64_t nrows, double *o, double *lse,
                   int nthreads) {
     if (!q || !k || !v || !rows || !o || !lse) return -1;
-    if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || nrows < 0) return -2;
+    if (B <= 0 || H <= 0 || Nq <= 0 || N <= 0 || d <= 0 || nrows < 0) return -2;
+    if (causal && Nq > N) return -2;
     if (!isfinite(scale)) return -3;
     if (nthreads <= 0) nthreads = oracle_default_threads();
     int64_t BH = (int64_t)B * H;
     for (int64_t r = 0; r < nrows; ++r) {
         if (rows[2 * r] < 0 || rows[2 * r] >= BH) return -4;
-        if (rows[2 * r + 1] < 0 || rows[2 * r + 1] >= N) return -4;
+        if (rows[2 * r + 1] < 0 || rows[2 * r + 1] >= Nq) return -4;
     }
     int64_t head_elems = (int64_t)N * d;
     double *K = (double *)malloc(sizeof(double) * (size_t)head_elems);
@@ -186,7 +200,7 @@ static int attend(const void *q, const void *k, const void *v, int kind, int B,
         }
         int nt = nmine < nthreads ? (int)nmine : nthreads;
         for (int t = 0; t < nt; ++t) {
-            job_t jb = {q, kind, K, V, bh, N, d, causal, scale, rows, mine, nmine,
+            job_t jb = {q, kind, K, V, bh, N, d, causal, scale, rows, mine, nmine, Nq,
                         t, nt, o, lse, 0, 0};
             jobs[t] = jb;
         }
@@ -218,7 +232,7 @@ int oracle_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      int B, int H, int N, int d, double scale, int causal,
                      const int64_t *rows, int64_t nrows, double *o, double *lse,
                      int nthreads) {
-    return attend(q, k, v, IN_BF16, B, H, N, d, scale, causal, rows, nrows, o,
+    return attend(q, k, v, IN_BF16, B, H, N, N, d, scale, causal, rows, nrows, o,
                   lse, nthreads);
 }
 
@@ -227,7 +241,27 @@ int oracle_attn_f64(const double *q, const double *k, const double *v, int B,
                     int H, int N, int d, double scale, int causal,
                     const int64_t *rows, int64_t nrows, double *o, double *lse,
                     int nthreads) {
-    return attend(q, k, v, IN_F64, B, H, N, d, scale, causal, rows, nrows, o,
+    return attend(q, k, v, IN_F64, B, H, N, N, d, scale, causal, rows, nrows, o,
+                  lse, nthreads);
+}
+
+/* Nq queries against Nk keys per head: q is [B, H, Nq, d], k and v are
+ * [B, H, Nk, d] (bf16 bit patterns); rows are (bh, i) with i < Nq; causal
+ * requires Nq <= Nk (the queries are the last Nq positions). */
+int oracle_attn_kv_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        int B, int H, int Nq, int Nk, int d, double scale,
+                        int causal, const int64_t *rows, int64_t nrows, double *o,
+                        double *lse, int nthreads) {
+    return attend(q, k, v, IN_BF16, B, H, Nq, Nk, d, scale, causal, rows, nrows, o,
+                  lse, nthreads);
+}
+
+/* Same with double inputs. */
+int oracle_attn_kv_f64(const double *q, const double *k, const double *v, int B,
+                       int H, int Nq, int Nk, int d, double scale, int causal,
+                       const int64_t *rows, int64_t nrows, double *o, double *lse,
+                       int nthreads) {
+    return attend(q, k, v, IN_F64, B, H, Nq, Nk, d, scale, causal, rows, nrows, o,
                   lse, nthreads);
 }
 
@@ -236,7 +270,7 @@ int oracle_attn_f64(const double *q, const double *k, const double *v, int B,
 int oracle_probs_f64(const double *q, const double *k, int N, int d,
                      double scale, int causal, int i, double *p) {
     if (!q || !k || !p || N <= 0 || d <= 0 || i < 0 || i >= N) return -1;
-    int nkeys = causal ? i + 1 : N;
+    int nkeys = allowed_keys(i, N, N, causal);
     double m, l;
     for (int j = 0; j < N; ++j) p[j] = 0.0;
     scores_row(q + (int64_t)i * d, k, nkeys, d, scale, p);

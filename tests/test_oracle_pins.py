@@ -206,3 +206,50 @@ def test_rejects_bad_rows():
         oracle.attention(q, k, v, 1.0, False, rows=np.array([[0, 4]]))
     with pytest.raises(RuntimeError):
         oracle.attention(q, k, v, float("nan"), False)
+
+
+# ----------------------------------------------------------------- Nq != Nk
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 9), (3, 11), (7, 7), (5, 16)])
+def test_kv_brute_force_vs_torch_softmax(Nq, Nk, causal):
+    # queries are the last Nq of Nk positions: causally query i sees keys
+    # j <= i + (Nk - Nq); brute force with torch's float64 softmax
+    B, H, d = 2, 2, 4
+    q = RNG.standard_normal((B, H, Nq, d))
+    k = RNG.standard_normal((B, H, Nk, d))
+    v = RNG.standard_normal((B, H, Nk, d))
+    o, lse = oracle.attention_kv(q, k, v, 0.45, causal)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    logits = torch.einsum("bhid,bhjd->bhij", tq, tk) * 0.45
+    if causal:
+        i = torch.arange(Nq)[:, None]
+        j = torch.arange(Nk)[None, :]
+        logits = logits.masked_fill(j > i + (Nk - Nq), float("-inf"))
+    ref = torch.softmax(logits, dim=-1) @ tv
+    assert np.abs(o - ref.numpy().reshape(-1, d)).max() <= 1e-12
+    assert np.abs(lse - torch.logsumexp(logits, -1).numpy().reshape(-1)).max() <= 1e-12
+
+
+def test_kv_queries_are_the_last_rows_of_full_attention():
+    # the decode shape is the tail of the square problem: the last Nq rows of
+    # causal attention over Nk positions equal Nq queries against Nk keys
+    B, H, Nk, Nq, d = 1, 3, 40, 6, 5
+    q_full = RNG.standard_normal((B, H, Nk, d))
+    k = RNG.standard_normal((B, H, Nk, d))
+    v = RNG.standard_normal((B, H, Nk, d))
+    o_full, lse_full = oracle.attention(q_full, k, v, 0.3, True)
+    o_tail, lse_tail = oracle.attention_kv(q_full[:, :, Nk - Nq:], k, v, 0.3, True)
+    sel = np.concatenate([np.arange(bh * Nk + Nk - Nq, (bh + 1) * Nk) for bh in range(B * H)])
+    assert np.array_equal(o_tail, o_full[sel]) and np.array_equal(lse_tail, lse_full[sel])
+    # with Nq = Nk the two entry points are the same function
+    o2, lse2 = oracle.attention_kv(q_full, k, v, 0.3, True)
+    assert np.array_equal(o2, o_full) and np.array_equal(lse2, lse_full)
+
+
+def test_kv_single_query_causal_sees_every_key():
+    q = RNG.standard_normal((1, 2, 1, 4))
+    k = RNG.standard_normal((1, 2, 13, 4))
+    v = RNG.standard_normal((1, 2, 13, 4))
+    o_c, l_c = oracle.attention_kv(q, k, v, 0.5, True)
+    o_n, l_n = oracle.attention_kv(q, k, v, 0.5, False)
+    assert np.array_equal(o_c, o_n) and np.array_equal(l_c, l_n)
