@@ -16,7 +16,8 @@ import os
 import threading
 
 __all__ = [
-    "AttnError", "lib", "attn_fwd", "attn_fwd_naive", "naive_workspace_bytes",
+    "AttnError", "lib", "attn_fwd", "attn_fwd_kv", "kv_num_splits", "kv_workspace_bytes",
+    "attn_fwd_naive", "naive_workspace_bytes",
     "last_device_error", "status_string", "selftest_wait_timeout", "abi",
     "NOALLOC_SCRATCH_BYTES",
 ]
@@ -58,6 +59,12 @@ def lib() -> ctypes.CDLL:
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.attn_fwd.restype = i
+        L.attn_fwd_kv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
+        L.attn_fwd_kv.restype = i
+        L.attn_fwd_kv_num_splits.argtypes = [i, i, i, i, i]
+        L.attn_fwd_kv_num_splits.restype = i
+        L.attn_fwd_kv_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        L.attn_fwd_kv_workspace_bytes.restype = sz
         L.attn_fwd_naive_workspace_bytes.argtypes = [i, i, i]
         L.attn_fwd_naive_workspace_bytes.restype = sz
         L.attn_fwd_naive.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
@@ -82,6 +89,20 @@ class abi:
     @staticmethod
     def attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream) -> int:
         return lib().attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream)
+
+    @staticmethod
+    def attn_fwd_kv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, num_splits, ws, ws_bytes,
+                    stream) -> int:
+        return lib().attn_fwd_kv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, num_splits, ws,
+                                 ws_bytes, stream)
+
+    @staticmethod
+    def attn_fwd_kv_num_splits(B, H, Nq, Nk, d) -> int:
+        return lib().attn_fwd_kv_num_splits(B, H, Nq, Nk, d)
+
+    @staticmethod
+    def attn_fwd_kv_workspace_bytes(B, H, Nq, Nk, d, num_splits) -> int:
+        return int(lib().attn_fwd_kv_workspace_bytes(B, H, Nq, Nk, d, num_splits))
 
     @staticmethod
     def attn_fwd_naive(q, k, v, o, lse, B, H, N, d, scale, causal, ws, ws_bytes, stream) -> int:
@@ -155,6 +176,48 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
                       B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def kv_num_splits(B: int, H: int, Nq: int, Nk: int, d: int) -> int:
+    """Split count attn_fwd_kv picks for num_splits=0 on the current device."""
+    st = abi.attn_fwd_kv_num_splits(B, H, Nq, Nk, d)
+    if st < 1:
+        raise AttnError(st, "attn_fwd_kv_num_splits")
+    return st
+
+
+def kv_workspace_bytes(B: int, H: int, Nq: int, Nk: int, d: int, num_splits: int = 0) -> int:
+    return abi.attn_fwd_kv_workspace_bytes(B, H, Nq, Nk, d, num_splits)
+
+
+def attn_fwd_kv(q, k, v, o=None, lse=None, scale=None, causal=False, num_splits=0,
+                workspace=None, stream=None):
+    """Nq query rows against Nk keys: q [B,H,Nq,d], k and v [B,H,Nk,d] (CUDA bf16,
+    contiguous). Causal alignment is bottom-right (query i sees keys j <= i + Nk - Nq).
+    num_splits=0 lets the library choose. Returns (o [B,H,Nq,d] bf16, lse [B,H,Nq] fp32)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous bf16 [B, H, N, d] tensor")
+    if k.shape != v.shape or k.shape[:2] != q.shape[:2] or k.shape[3] != q.shape[3]:
+        raise ValueError("q [B, H, Nq, d] and k, v [B, H, Nk, d] expected")
+    B, H, Nq, d = (int(x) for x in q.shape)
+    Nk = int(k.shape[2])
+    o, lse = _outputs(q, o, lse)
+    need = kv_workspace_bytes(B, H, Nq, Nk, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = abi.attn_fwd_kv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                         B, H, Nq, Nk, d, scale, int(bool(causal)), int(num_splits), ws_ptr,
+                         ws_bytes, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_kv")
     return o, lse
 
 

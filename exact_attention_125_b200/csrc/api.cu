@@ -76,6 +76,103 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+int validate_kv(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                int B, int H, int Nq, int Nk, int d, float scale, int causal) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return ATTN_ERR_SHAPE;
+  if (static_cast<long long>(B) * H * Nq > INT_MAX || static_cast<long long>(B) * H * Nk > INT_MAX)
+    return ATTN_ERR_SHAPE;
+  if (d != 64 && d != 128) return ATTN_ERR_HEADDIM;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4))
+    return ATTN_ERR_ALIGN;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_SCALE;
+  if (causal != 0 && causal != 1) return ATTN_ERR_CAUSAL;
+  if (causal && Nq > Nk) return ATTN_ERR_SHAPE;
+  return ATTN_OK;
+}
+
+bool kv_shape_ok(int B, int H, int Nq, int Nk, int d) {
+  return B >= 1 && H >= 1 && Nq >= 1 && Nk >= 1 && (d == 64 || d == 128) &&
+         static_cast<long long>(B) * H * Nq <= INT_MAX && static_cast<long long>(B) * H * Nk <= INT_MAX;
+}
+
+int sm_count(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+// Requested split count -> effective plan; num_splits = 0 asks for the
+// automatic choice on the current device.
+int resolve_kv_plan(int B, int H, int Nq, int Nk, int num_splits, attn::KvPlan* plan) {
+  if (num_splits < 0 || num_splits > attn::kMaxKvSplits) return ATTN_ERR_SHAPE;
+  const int BH = B * H;
+  if (num_splits == 0) {
+    int st = check_device();
+    if (st != ATTN_OK) return st;
+    int sms = 0;
+    if ((st = sm_count(&sms)) != ATTN_OK) return st;
+    num_splits = attn::default_kv_splits(BH, Nq, Nk, sms);
+  }
+  *plan = attn::plan_kv(BH, Nq, Nk, num_splits);
+  return ATTN_OK;
+}
+
+}  // namespace
+
+int attn_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int Nq, int Nk, int d, float scale, int causal, int num_splits, void* workspace,
+                size_t workspace_bytes, attn_stream_t stream) {
+  int st = validate_kv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (num_splits < 0 || num_splits > attn::kMaxKvSplits) return ATTN_ERR_SHAPE;
+  // An explicit split count is checked against the workspace before the
+  // device is touched; the automatic one needs the device's SM count.
+  if (num_splits == 0 && (st = check_device()) != ATTN_OK) return st;
+  attn::KvPlan plan{};
+  if ((st = resolve_kv_plan(B, H, Nq, Nk, num_splits, &plan)) != ATTN_OK) return st;
+  const size_t need = attn::kv_workspace_bytes(B * H, Nq, d, plan.nsplit);
+  if (need > 0) {
+    if (!workspace) return ATTN_ERR_NULL;
+    if (!aligned(workspace, 256)) return ATTN_ERR_ALIGN;
+    if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  }
+  if ((st = check_device()) != ATTN_OK) return st;
+  attn::AttnKvArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.d = d;
+  a.scale = scale;
+  a.causal = causal;
+  return attn::launch_fused_kv(a, plan, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_kv_num_splits(int B, int H, int Nq, int Nk, int d) {
+  if (!kv_shape_ok(B, H, Nq, Nk, d)) return ATTN_ERR_SHAPE;
+  attn::KvPlan plan{};
+  const int st = resolve_kv_plan(B, H, Nq, Nk, 0, &plan);
+  return st != ATTN_OK ? st : plan.nsplit;
+}
+
+size_t attn_fwd_kv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits) {
+  if (!kv_shape_ok(B, H, Nq, Nk, d)) return 0;
+  attn::KvPlan plan{};
+  if (resolve_kv_plan(B, H, Nq, Nk, num_splits, &plan) != ATTN_OK) return 0;
+  return attn::kv_workspace_bytes(B * H, Nq, d, plan.nsplit);
+}
+
 size_t attn_fwd_naive_workspace_bytes(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return 0;
   const unsigned long long bh = static_cast<unsigned long long>(B) * H;

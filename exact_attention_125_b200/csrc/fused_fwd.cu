@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -91,6 +92,10 @@ struct Cfg {
   static constexpr int kNumBars = 1 + 2 * kStages + 6 + 1;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;  // tmem base, abort flag
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;   // + alignment slack
+  // kv path: (m, l) of every softmax thread, swapped between the two
+  // warpgroups when they took alternate KV tiles of one query tile
+  static constexpr int kXchOff = kMiscOff + 16;
+  static constexpr int kSmemBytesKv = kXchOff + 256 * 2 * 4 + 1024;
   __host__ __device__ static constexpr uint32_t col_s(int g) { return g == 0 ? 0u : 128u; }
   __host__ __device__ static constexpr uint32_t col_o(int g) { return 256u + (g == 0 ? 0u : uint32_t(D)); }
 };
@@ -99,16 +104,84 @@ struct FwdParams {
   void* o;
   float* lse;
   unsigned int* err;
-  int N, BH, nqb, T;
+  int N, BH, nqb, T;  // N = keys (and query rows of the square problem); T = KV tiles
   float scale_log2;
   int causal;
   uint64_t wait_limit_ns;
+  // kv path only (Nq query rows against N keys, KV range split across CTAs)
+  int Nq;
+  int offset;    // N - Nq: causally, query row i is sequence position i + offset
+  int nsplit;    // KV splits (1: O and lse written directly)
+  int tps;       // KV tiles per split
+  int alt;       // 1: one query tile per CTA, the two softmax warpgroups take alternate KV tiles
+  float* part_o;    // [nsplit][BH][Nq][D] fp32, normalised per split (nsplit > 1)
+  float* part_lse;  // [nsplit][BH][Nq] fp32 natural-log lse per split (nsplit > 1)
 };
 
+// What one CTA of the kv path works on.
+struct KvWork {
+  int split;
+  int kv_lo;  // first KV tile of the split
+  int na, nb; // KV tiles for softmax warpgroup a / b
+};
+
+// kv path: the (head, query block, KV split) of this CTA and the KV tiles each
+// softmax warpgroup takes. Cheap integer arithmetic on blockIdx and the
+// parameters, so the softmax warps recompute it for their epilogue instead of
+// keeping it in registers through the main loop.
+__device__ __forceinline__ KvWork kv_work_of(const FwdParams& p, int& bh, int& q0) {
+  KvWork kw{0, 0, 0, 0};
+  // (bh, split, query block), query blocks fastest; a block is one query
+  // tile when alt, else two.
+  const int per_bh = p.nqb * p.nsplit;
+  bh = blockIdx.x / per_bh;
+  const int rem = blockIdx.x % per_bh;
+  kw.split = rem / p.nqb;
+  const int r = rem % p.nqb;
+  const int qblk = p.causal ? (p.nqb - 1 - r) : r;
+  q0 = qblk * (p.alt ? kTileRows : kBlockRows);
+  kw.kv_lo = kw.split * p.tps;
+  const int kv_hi = min(p.T, kw.kv_lo + p.tps);
+  // KV tiles up to the last one that some row of the tile starting at r0 sees
+  auto need = [&](int r0) -> int {
+    if (r0 >= p.Nq) return 0;
+    if (!p.causal) return p.T;
+    const int r1 = min(r0 + kTileRows - 1, p.Nq - 1);
+    return min(p.T, (r1 + p.offset) / kTileRows + 1);
+  };
+  if (p.alt) {
+    const int n = max(0, min(kv_hi, need(q0)) - kw.kv_lo);
+    kw.na = (n + 1) / 2;
+    kw.nb = n / 2;
+  } else {
+    kw.na = max(0, min(kv_hi, need(q0)) - kw.kv_lo);
+    kw.nb = max(0, min(kv_hi, need(q0 + kTileRows)) - kw.kv_lo);
+  }
+  return kw;
+}
+
+// Stores 32 consecutive output columns of one row: fp32 (a split's partial
+// result) or bf16 (the final O).
 template <int D>
+__device__ __forceinline__ void store_row_chunk(const FwdParams& p, bool partial, size_t row_index,
+                                                int col, const float (&v)[32]) {
+  if (partial) {
+    float4* dst = reinterpret_cast<float4*>(p.part_o + row_index * D + col);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row_index * D + col);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      dst[u] = make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                          pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+  }
+}
+
+template <int D, bool kKV>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, uint32_t bars,
                                              int bh, int q0, int n_kv, int g,
-                                             const Watchdog& wd) {
+                                             const Watchdog& wd, int kv_lo) {
   using C = Cfg<D>;
   const int warp = threadIdx.x / 32;
   const int tid = threadIdx.x % 128;
@@ -118,7 +191,9 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
   const uint32_t bar_s_full = bars + 8u * (1 + 2 * C::kStages + g);
   const uint32_t bar_p_ready = bars + 8u * (1 + 2 * C::kStages + 2 + g);
   const uint32_t bar_o_final = bars + 8u * (1 + 2 * C::kStages + 4 + g);
-  const int row_start = q0 + kTileRows * g;
+  // kv path with alternate KV tiles: both warpgroups hold the same query rows
+  const bool alt = kKV && p.alt;
+  const int row_start = alt ? q0 : q0 + kTileRows * g;
   const int row = row_start + tid;
   const float c = p.scale_log2;
 
@@ -131,11 +206,18 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     uint32_t sr[128];
     tmem_ld_x128_wait(tS, sr);
 
-    const int col0 = j * kTileRows;
-    const bool need_mask = (p.causal && col0 + kTileRows - 1 > row_start) || (col0 + kTileRows > p.N);
+    bool need_mask;
+    int col0;
+    if constexpr (kKV) {
+      col0 = (kv_lo + (alt ? 2 * j + g : j)) * kTileRows;
+      need_mask = (p.causal && col0 + kTileRows - 1 > row_start + p.offset) || (col0 + kTileRows > p.N);
+    } else {
+      col0 = j * kTileRows;
+      need_mask = (p.causal && col0 + kTileRows - 1 > row_start) || (col0 + kTileRows > p.N);
+    }
     if (need_mask) {
       int lim = p.N - 1 - col0;
-      if (p.causal) lim = min(lim, row - col0);
+      if (p.causal) lim = min(lim, row + (kKV ? p.offset : 0) - col0);
 #pragma unroll
       for (int cc = 0; cc < 128; ++cc)
         if (cc > lim) sr[cc] = 0xff800000u;  // -inf
@@ -199,32 +281,120 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     tc_fence_before_sync();
     mbar_arrive(bar_p_ready);
   }
-  if (ok) ok = warp_wait(bar_o_final, 0, wd);
-  if (!ok) return;
-  tc_fence_after_sync();
+  if constexpr (!kKV) {
+    if (ok) ok = warp_wait(bar_o_final, 0, wd);
+    if (!ok) return;
+    tc_fence_after_sync();
 
-  // Epilogue: O / l -> bf16, lse in natural log.
-  const float inv_l = 1.0f / l_run;
-  const bool valid = row < p.N;
-  uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
-                                         (static_cast<size_t>(bh) * p.N + row) * D);
+    // Epilogue: O / l -> bf16, lse in natural log.
+    const float inv_l = 1.0f / l_run;
+    const bool valid = row < p.N;
+    uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
+                                           (static_cast<size_t>(bh) * p.N + row) * D);
 #pragma unroll
-  for (int ch = 0; ch < D / 32; ++ch) {
-    uint32_t orr[32];
-    tmem_ld_x32_wait(tO + ch * 32, orr);
-    uint32_t w[16];
+    for (int ch = 0; ch < D / 32; ++ch) {
+      uint32_t orr[32];
+      tmem_ld_x32_wait(tO + ch * 32, orr);
+      uint32_t w[16];
 #pragma unroll
-    for (int u = 0; u < 16; ++u)
-      w[u] = pack_bf16x2(__uint_as_float(orr[2 * u]) * inv_l, __uint_as_float(orr[2 * u + 1]) * inv_l);
-    if (valid) {
+      for (int u = 0; u < 16; ++u)
+        w[u] = pack_bf16x2(__uint_as_float(orr[2 * u]) * inv_l, __uint_as_float(orr[2 * u + 1]) * inv_l);
+      if (valid) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        orow[ch * 4 + u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        for (int u = 0; u < 4; ++u)
+          orow[ch * 4 + u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
     }
-  }
-  if (valid) {
-    const float m_fin = (m_run == -INFINITY) ? 0.0f : m_run;
-    p.lse[static_cast<size_t>(bh) * p.N + row] = (m_fin + __log2f(l_run)) * 0.69314718055994531f;
+    if (valid) {
+      const float m_fin = (m_run == -INFINITY) ? 0.0f : m_run;
+      p.lse[static_cast<size_t>(bh) * p.N + row] = (m_fin + __log2f(l_run)) * 0.69314718055994531f;
+    }
+  } else {
+    // A row that saw no unmasked key in this KV range (possible only when the
+    // range is a split that starts past the row's causal limit): l = 0, which
+    // gives O = 0 and lse = -inf, the neutral element of the combine.
+    if (m_run == -INFINITY) l_run = 0.0f;
+    int bh_unused, q0_unused;
+    const KvWork kw = kv_work_of(p, bh_unused, q0_unused);
+    const bool valid = row < p.Nq;
+    const bool partial = p.nsplit > 1;
+    const size_t row_index =
+        (partial ? static_cast<size_t>(kw.split) * p.BH + bh : static_cast<size_t>(bh)) * p.Nq + row;
+    float* lse_dst = partial ? p.part_lse : p.lse;
+    const uint32_t bar_o_final0 = bars + 8u * (1 + 2 * C::kStages + 4);
+    if (!alt) {
+      if (ok && n_kv > 0) ok = warp_wait(bar_o_final, 0, wd);
+      if (!ok) return;
+      tc_fence_after_sync();
+      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float v[32];
+        if (n_kv > 0) {
+          uint32_t orr[32];
+          tmem_ld_x32_wait(tO + ch * 32, orr);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(orr[u]) * inv_l;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = 0.0f;
+        }
+        if (valid) store_row_chunk<D>(p, partial, row_index, ch * 32, v);
+      }
+      if (valid)
+        lse_dst[row_index] = l_run > 0.0f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    } else {
+      // Both warpgroups hold the same rows: O = (O_a 2^(m_a-m) + O_b 2^(m_b-m)) /
+      // (l_a 2^(m_a-m) + l_b 2^(m_b-m)) with m = max(m_a, m_b). Each warpgroup
+      // waits for both accumulators, swaps (m, l) through shared memory and
+      // writes half of the columns. Every softmax thread reaches the named
+      // barrier, also after a failed wait, and all leave together if any wait
+      // failed (a failed wait always sets the CTA's abort flag).
+      if (ok && kw.na > 0) ok = warp_wait(bar_o_final0, 0, wd);
+      if (ok && kw.nb > 0) ok = warp_wait(bar_o_final0 + 8u, 0, wd);
+      extern __shared__ uint8_t smem_raw[];
+      const uint32_t raw = smem_u32(smem_raw);
+      float* xch = reinterpret_cast<float*>(smem_raw + (((raw + 1023u) & ~1023u) - raw) + C::kXchOff);
+      xch[2 * (128 * g + tid)] = m_run;
+      xch[2 * (128 * g + tid) + 1] = l_run;
+      named_barrier_sync(1, 256);
+      if (*wd.abort) return;
+      tc_fence_after_sync();
+      const float m_o = xch[2 * (128 * (1 - g) + tid)];
+      const float l_o = xch[2 * (128 * (1 - g) + tid) + 1];
+      const float m_a = g == 0 ? m_run : m_o, l_a = g == 0 ? l_run : l_o;
+      const float m_b = g == 0 ? m_o : m_run, l_b = g == 0 ? l_o : l_run;
+      const float m = fmaxf(m_a, m_b);
+      const float sa = l_a > 0.0f ? ex2_approx(m_a - m) : 0.0f;
+      const float sb = l_b > 0.0f ? ex2_approx(m_b - m) : 0.0f;
+      const float L = l_a * sa + l_b * sb;
+      const float inv_L = L > 0.0f ? 1.0f / L : 0.0f;
+      const float wa = sa * inv_L, wb = sb * inv_L;
+      const uint32_t tOa = tmem + lane_base + C::col_o(0);
+      const uint32_t tOb = tmem + lane_base + C::col_o(1);
+#pragma unroll
+      for (int ch = 0; ch < D / 64; ++ch) {
+        const int col = g * (D / 2) + ch * 32;
+        float v[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = 0.0f;
+        if (kw.na > 0) {
+          uint32_t orr[32];
+          tmem_ld_x32_wait(tOa + col, orr);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(orr[u]) * wa;
+        }
+        if (kw.nb > 0) {
+          uint32_t orr[32];
+          tmem_ld_x32_wait(tOb + col, orr);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = fmaf(__uint_as_float(orr[u]), wb, v[u]);
+        }
+        if (valid) store_row_chunk<D>(p, partial, row_index, col, v);
+      }
+      if (valid && g == 0)
+        lse_dst[row_index] = L > 0.0f ? (m + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
   }
 }
 
@@ -363,7 +533,192 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   drain_wait(bar_mma_done, 0, wd);
 }
 
+// kv path producer. Query rows q0.. (one tile when alt, else two), then K/V
+// tiles of the CTA's range [kv_lo, kv_lo + n) in two-slot units:
+//   shared (both query tiles see every KV tile): unit 0 = K_0, unit u >= 1 =
+//     (V_{u-1}, K_u), unit n = V_{n-1} only;
+//   alt (warpgroup a takes KV tiles 0, 2, 4, ..., b takes 1, 3, 5, ...):
+//     unit 0 = (K_0, K_1), unit u >= 1 = (V_{u-1}, K_{u+1}).
+// Tile indices are relative to kv_lo.
 template <int D>
+__device__ __forceinline__ void producer_role_kv(const CUtensorMap* tq, const CUtensorMap* tk,
+                                                 const CUtensorMap* tv, uint32_t base,
+                                                 uint32_t bars, int bh, int q0, int kv_lo, int n,
+                                                 bool alt, bool kv_reuse, const Watchdog& wd) {
+  using C = Cfg<D>;
+  if (n == 0) return;
+  const uint32_t sQ = base + C::kQOff;
+  const uint32_t sRing = base + C::kRingOff;
+  const uint32_t bar_q = bars;
+  const uint64_t pol_q = l2_policy_evict_first();
+  // with one query block per head every KV tile is read by exactly one CTA
+  const uint64_t pol_kv = kv_reuse ? l2_policy_evict_last() : l2_policy_evict_first();
+  const int nq = alt ? 1 : 2;
+
+  mbar_arrive_expect_tx(bar_q, nq * C::kTileBytes);
+  for (int g = 0; g < nq; ++g)
+#pragma unroll
+    for (int a = 0; a < C::kAtoms; ++a)
+      tma_load_3d_hint(sQ + g * C::kTileBytes + a * C::kAtomBytes, tq, bar_q, a * 64,
+                       q0 + g * kTileRows, bh, pol_q);
+
+  int u = 0;
+  for (; u <= n; ++u) {
+    const int us = u % C::kUnits;
+    const uint32_t ph = (u / C::kUnits) & 1;
+    const uint32_t bar_full = bars + 8u * (1 + us);
+    const uint32_t bar_empty = bars + 8u * (1 + C::kStages + us);
+    if (!wait_one(bar_empty, ph ^ 1u, wd)) break;
+    const CUtensorMap* map0 = nullptr;  // first slot of the unit
+    const CUtensorMap* map1 = nullptr;  // second slot
+    int t0 = 0, t1 = 0;
+    if (alt) {
+      if (u == 0) {
+        map0 = tk;
+        t0 = 0;
+        if (n > 1) map1 = tk, t1 = 1;
+      } else {
+        map0 = tv;
+        t0 = u - 1;
+        if (u + 1 < n) map1 = tk, t1 = u + 1;
+      }
+    } else {
+      if (u >= 1) map0 = tv, t0 = u - 1;
+      if (u < n) map1 = tk, t1 = u;
+    }
+    mbar_arrive_expect_tx(bar_full, (int(map0 != nullptr) + int(map1 != nullptr)) * C::kTileBytes);
+    if (map0) {
+#pragma unroll
+      for (int a = 0; a < C::kAtoms; ++a)
+        tma_load_3d_hint(sRing + (2 * us) * C::kTileBytes + a * C::kAtomBytes, map0, bar_full,
+                         a * 64, (kv_lo + t0) * kTileRows, bh, pol_kv);
+    }
+    if (map1) {
+#pragma unroll
+      for (int a = 0; a < C::kAtoms; ++a)
+        tma_load_3d_hint(sRing + (2 * us + 1) * C::kTileBytes + a * C::kAtomBytes, map1, bar_full,
+                         a * 64, (kv_lo + t1) * kTileRows, bh, pol_kv);
+    }
+  }
+  drain_wait(bar_q, 0, wd);
+  for (int w = (u > C::kUnits ? u - C::kUnits : 0); w < u; ++w)
+    drain_wait(bars + 8u * (1 + w % C::kUnits), (w / C::kUnits) & 1, wd);
+}
+
+// kv path MMA issuer; the unit layout is the one producer_role_kv loads.
+template <int D>
+__device__ __forceinline__ void mma_role_kv(uint32_t tmem, uint32_t base, uint32_t bars, int na,
+                                            int nb, bool alt, const Watchdog& wd) {
+  using C = Cfg<D>;
+  const uint32_t sQ = base + C::kQOff;
+  const uint32_t sRing = base + C::kRingOff;
+  const uint32_t bar_q = bars;
+  const uint32_t bar_s_full0 = bars + 8u * (1 + 2 * C::kStages);
+  const uint32_t bar_p_ready0 = bar_s_full0 + 16u;
+  const uint32_t bar_o_final0 = bar_s_full0 + 32u;
+  const uint32_t bar_mma_done = bar_s_full0 + 48u;
+  constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+
+  auto par_of = [](int u) { return static_cast<uint32_t>((u / C::kUnits) & 1); };
+  auto full_bar = [&](int u) { return bars + 8u * (1 + u % C::kUnits); };
+  auto empty_bar = [&](int u) { return bars + 8u * (1 + C::kStages + u % C::kUnits); };
+  auto slot0 = [](int u) { return 2 * (u % C::kUnits); };
+  auto slot1 = [](int u) { return 2 * (u % C::kUnits) + 1; };
+
+  // S_g = Q_qt K^T into tile g's S columns
+  auto issue_qk = [&](int g, int qt, int slot) {
+    const uint32_t a0 = sQ + qt * C::kTileBytes;
+    const uint32_t b0 = sRing + slot * C::kTileBytes;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * C::kAtomBytes + (kk & 3) * 32;
+      mma_ss(tmem + C::col_s(g), sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
+             idesc_qk, kk > 0 ? 1u : 0u);
+    }
+  };
+  auto issue_pv = [&](int g, int slot, bool accumulate) {
+    const uint32_t b0 = sRing + slot * C::kTileBytes;
+#pragma unroll
+    for (int kk = 0; kk < kTileRows / 16; ++kk)
+      mma_ts(tmem + C::col_o(g), tmem + C::col_s(g) + kk * 8,
+             sdesc_sw128(b0 + kk * 2048, C::kAtomBytes, 1024), idesc_pv,
+             (accumulate || kk > 0) ? 1u : 0u);
+  };
+
+  const int n = alt ? na + nb : max(na, nb);
+  if (n > 0) {
+    bool ok = wait_one(bar_q, 0, wd) && wait_one(full_bar(0), par_of(0), wd);
+    if (ok) {
+      tc_fence_after_sync();
+      if (alt) {
+        issue_qk(0, 0, slot0(0));
+        mma_commit(bar_s_full0);
+        if (nb > 0) {
+          issue_qk(1, 0, slot1(0));
+          mma_commit(bar_s_full0 + 8u);
+        }
+      } else {
+        if (na > 0) {
+          issue_qk(0, 0, slot1(0));
+          mma_commit(bar_s_full0);
+        }
+        if (nb > 0) {
+          issue_qk(1, 1, slot1(0));
+          mma_commit(bar_s_full0 + 8u);
+        }
+      }
+      mma_commit(empty_bar(0));
+    }
+    if (alt) {
+      // unit u: V_{u-1} for warpgroup g = (u-1) % 2 (its step i = (u-1) / 2),
+      // and K_{u+1}, that warpgroup's next KV tile
+      for (int u = 1; ok && u <= n; ++u) {
+        const int g = (u - 1) & 1;
+        const int i = (u - 1) >> 1;
+        if (!(ok = wait_one(full_bar(u), par_of(u), wd))) break;
+        if (!(ok = wait_one(bar_p_ready0 + 8u * g, i & 1, wd))) break;
+        tc_fence_after_sync();
+        issue_pv(g, slot0(u), i > 0);
+        if (u + 1 < n) {
+          issue_qk(g, 0, slot1(u));
+          mma_commit(bar_s_full0 + 8u * g);
+        } else {
+          mma_commit(bar_o_final0 + 8u * g);
+        }
+        mma_commit(empty_bar(u));
+      }
+    } else {
+      for (int j = 0; ok && j < n; ++j) {
+        const int u = j + 1;  // V_j and K_{j+1}
+        if (!(ok = wait_one(full_bar(u), par_of(u), wd))) break;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int ng = g == 0 ? na : nb;
+          if (j < ng) {
+            if (!(ok = wait_one(bar_p_ready0 + 8u * g, j & 1, wd))) break;
+            tc_fence_after_sync();
+            issue_pv(g, slot0(u), j > 0);
+            if (j + 1 < ng) {
+              issue_qk(g, g, slot1(u));
+              mma_commit(bar_s_full0 + 8u * g);
+            } else {
+              mma_commit(bar_o_final0 + 8u * g);
+            }
+          }
+        }
+        if (!ok) break;
+        mma_commit(empty_bar(u));
+      }
+    }
+  }
+  mma_commit(bar_mma_done);
+  drain_wait(bar_mma_done, 0, wd);
+}
+
+// kD: head dimension. kKV: the kv path (Nq query rows against N keys, the
+// KV range of each head split across CTAs); false: the square problem.
+template <int D, bool kKV>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                           const __grid_constant__ CUtensorMap tmap_k,
@@ -382,12 +737,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Work unit: heads are the slow index so co-resident CTAs share K/V in L2;
   // with causal masking the heaviest query blocks go first.
-  const int bh = blockIdx.x / p.nqb;
-  const int r = blockIdx.x % p.nqb;
-  const int qblk = p.causal ? (p.nqb - 1 - r) : r;
-  const int q0 = qblk * kBlockRows;
-  const int na = p.causal ? min(p.T, q0 / kTileRows + 1) : p.T;
-  const int nb = p.causal ? min(p.T, q0 / kTileRows + 2) : p.T;
+  int bh, q0, na, nb;
+  KvWork kw{0, 0, 0, 0};
+  if constexpr (!kKV) {
+    bh = blockIdx.x / p.nqb;
+    const int r = blockIdx.x % p.nqb;
+    const int qblk = p.causal ? (p.nqb - 1 - r) : r;
+    q0 = qblk * kBlockRows;
+    na = p.causal ? min(p.T, q0 / kTileRows + 1) : p.T;
+    nb = p.causal ? min(p.T, q0 / kTileRows + 2) : p.T;
+  } else {
+    kw = kv_work_of(p, bh, q0);
+    na = kw.na;
+    nb = kw.nb;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bars, 1);
@@ -424,13 +787,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
     const int g = warp / 4;
-    softmax_role<D>(p, tmem, bars, bh, q0, g == 0 ? na : nb, g, wd);
+    softmax_role<D, kKV>(p, tmem, bars, bh, q0, g == 0 ? na : nb, g, wd, kw.kv_lo);
   } else {
     regs_decrease<kRegsOther>();
-    if (warp == kProducerWarp) {
-      if (lane == 0) producer_role<D>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
-    } else if (warp == kMmaWarp) {
-      if (lane == 0) mma_role<D>(tmem, base, bars, na, nb, wd);
+    if constexpr (!kKV) {
+      if (warp == kProducerWarp) {
+        if (lane == 0) producer_role<D>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
+      } else if (warp == kMmaWarp) {
+        if (lane == 0) mma_role<D>(tmem, base, bars, na, nb, wd);
+      }
+    } else {
+      const bool alt = p.alt != 0;
+      if (warp == kProducerWarp) {
+        if (lane == 0)
+          producer_role_kv<D>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, kw.kv_lo,
+                              alt ? na + nb : max(na, nb), alt, p.nqb > 1, wd);
+      } else if (warp == kMmaWarp) {
+        if (lane == 0) mma_role_kv<D>(tmem, base, bars, na, nb, alt, wd);
+      }
     }
   }
   __syncwarp();
@@ -527,19 +901,117 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream) {
   p.wait_limit_ns = kWaitLimitNs;
   const long long grid = static_cast<long long>(p.nqb) * BH;
   if (grid > 0x7fffffffLL) return ATTN_ERR_SHAPE;
-  if (cudaFuncSetAttribute(fused_attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::kSmemBytes) != cudaSuccess)
+  auto kernel = fused_attn_fwd_kernel<D, false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
     return ATTN_ERR_CUDA;
   // The register split inside the kernel assumes this exact allocation.
   cudaFuncAttributes fa{};
-  if (cudaFuncGetAttributes(&fa, fused_attn_fwd_kernel<D>) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
   if (fa.numRegs != kRegsAtLaunch || fa.maxThreadsPerBlock < kThreads) return ATTN_ERR_LAUNCH;
-  fused_attn_fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
-      mq, mk, mv, p);
+  kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
+// ------------------------------------------------------------ kv path host
+
+template <int D>
+int launch_fused_kv_d(const AttnKvArgs& a, const KvPlan& plan, void* workspace,
+                      cudaStream_t stream) {
+  using C = Cfg<D>;
+  const int BH = a.B * a.H;
+  CUtensorMap mq, mk, mv;
+  if (!encode_qkv_map(&mq, a.q, BH, a.Nq, D) || !encode_qkv_map(&mk, a.k, BH, a.Nk, D) ||
+      !encode_qkv_map(&mv, a.v, BH, a.Nk, D))
+    return ATTN_ERR_CUDA;
+  unsigned int* err = device_error_word();
+  if (!err) return ATTN_ERR_CUDA;
+  FwdParams p{};
+  p.o = a.o;
+  p.lse = a.lse;
+  p.err = err;
+  p.N = a.Nk;
+  p.BH = BH;
+  p.nqb = plan.nqb;
+  p.T = plan.T;
+  p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
+  p.causal = a.causal;
+  p.wait_limit_ns = kWaitLimitNs;
+  p.Nq = a.Nq;
+  p.offset = a.Nk - a.Nq;
+  p.nsplit = plan.nsplit;
+  p.tps = plan.tps;
+  p.alt = plan.alt;
+  if (plan.nsplit > 1) {
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          kv_partial_o_bytes(BH, a.Nq, D, plan.nsplit));
+  }
+  const long long grid = static_cast<long long>(plan.nqb) * plan.nsplit * BH;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+  auto kernel = fused_attn_fwd_kernel<D, true>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytesKv) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (fa.numRegs != kRegsAtLaunch || fa.maxThreadsPerBlock < kThreads) return ATTN_ERR_LAUNCH;
+  kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytesKv, stream>>>(mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (plan.nsplit > 1)
+    return launch_lse_combine(p.part_o, p.part_lse, a.o, a.lse, BH * a.Nq, D, plan.nsplit, stream);
+  return ATTN_OK;
+}
+
 }  // namespace
+
+KvPlan plan_kv(int BH, int Nq, int Nk, int num_splits) {
+  KvPlan pl{};
+  pl.T = (Nk + kTileRows - 1) / kTileRows;
+  pl.alt = Nq <= kTileRows ? 1 : 0;
+  pl.nqb = (Nq + (pl.alt ? kTileRows : kBlockRows) - 1) / (pl.alt ? kTileRows : kBlockRows);
+  const int s = std::max(1, std::min(num_splits, pl.T));
+  pl.tps = (pl.T + s - 1) / s;
+  pl.nsplit = (pl.T + pl.tps - 1) / pl.tps;  // no empty split
+  (void)BH;
+  return pl;
+}
+
+int default_kv_splits(int BH, int Nq, int Nk, int sms) {
+  const KvPlan one = plan_kv(BH, Nq, Nk, 1);
+  const long long base = static_cast<long long>(BH) * one.nqb;
+  if (sms < 1 || base >= sms) return 1;
+  // At least kMinTilesPerSplit KV tiles per CTA keeps the per-CTA start-up
+  // (Q load, pipeline fill, epilogue) small against its streaming time.
+  constexpr int kMinTilesPerSplit = 8;
+  const int max_s = std::max(1, std::min(kMaxKvSplits, one.T / kMinTilesPerSplit));
+  auto eff = [&](int s) {
+    const long long n = base * plan_kv(BH, Nq, Nk, s).nsplit;
+    const long long waves = (n + sms - 1) / sms;
+    return static_cast<double>(n) / static_cast<double>(waves * sms);
+  };
+  double best = 0.0;
+  for (int s = 1; s <= max_s; ++s) best = std::max(best, eff(s));
+  // the fewest splits within 15% of the best wave efficiency
+  for (int s = 1; s <= max_s; ++s)
+    if (eff(s) >= 0.85 * best) return plan_kv(BH, Nq, Nk, s).nsplit;
+  return 1;
+}
+
+size_t kv_partial_o_bytes(int BH, int Nq, int d, int nsplit) {
+  const size_t b = static_cast<size_t>(nsplit) * BH * Nq * d * sizeof(float);
+  return (b + 255) & ~static_cast<size_t>(255);
+}
+
+size_t kv_workspace_bytes(int BH, int Nq, int d, int nsplit) {
+  if (nsplit <= 1) return 0;
+  return kv_partial_o_bytes(BH, Nq, d, nsplit) + static_cast<size_t>(nsplit) * BH * Nq * sizeof(float);
+}
+
+int launch_fused_kv(const AttnKvArgs& a, const KvPlan& plan, void* workspace, cudaStream_t stream) {
+  return a.d == 128 ? launch_fused_kv_d<128>(a, plan, workspace, stream)
+                    : launch_fused_kv_d<64>(a, plan, workspace, stream);
+}
 
 int launch_fused(const AttnArgs& a, cudaStream_t stream) {
   return a.d == 128 ? launch_fused_d<128>(a, stream) : launch_fused_d<64>(a, stream);

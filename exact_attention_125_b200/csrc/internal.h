@@ -22,6 +22,44 @@ struct AttnArgs {
 // Fused tcgen05 path (fused_fwd.cu). Arguments already validated.
 int launch_fused(const AttnArgs& a, cudaStream_t stream);
 
+// kv path: Nq query rows against Nk keys per head.
+struct AttnKvArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int B, H, Nq, Nk, d;
+  float scale;
+  int causal;
+};
+
+// How the kv path cuts the work: T KV tiles of 128 keys, tps tiles per split,
+// nsplit splits (none empty), nqb query blocks per head; alt = 1 when Nq <= 128
+// (one query tile per CTA, its two softmax warpgroups on alternate KV tiles).
+struct KvPlan {
+  int T, tps, nsplit, alt, nqb;
+};
+
+constexpr int kMaxKvSplits = 256;
+
+// Plan for a requested split count (clamped to [1, T]).
+KvPlan plan_kv(int BH, int Nq, int Nk, int num_splits);
+// Split count the library picks for a GPU with `sms` multiprocessors.
+int default_kv_splits(int BH, int Nq, int Nk, int sms);
+// Bytes of the fp32 partial-O block (rounded up to 256) and of the whole
+// workspace (partial O, then partial lse) for nsplit splits; 0 when nsplit <= 1.
+size_t kv_partial_o_bytes(int BH, int Nq, int d, int nsplit);
+size_t kv_workspace_bytes(int BH, int Nq, int d, int nsplit);
+// Fused kernel over the plan, then the combine when plan.nsplit > 1.
+int launch_fused_kv(const AttnKvArgs& a, const KvPlan& plan, void* workspace, cudaStream_t stream);
+
+// LSE-weighted combine of nsplit partial results (combine.cu): for each of
+// `rows` rows, O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max lse),
+// lse = max lse + log sum_s w_s; O written as bf16.
+int launch_lse_combine(const float* part_o, const float* part_lse, void* o, float* lse, int rows,
+                       int d, int nsplit, cudaStream_t stream);
+
 // Unfused three-kernel path (naive.cu). Arguments already validated.
 int launch_naive(const AttnArgs& a, void* workspace, cudaStream_t stream);
 

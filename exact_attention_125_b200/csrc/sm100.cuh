@@ -142,6 +142,12 @@ __device__ __forceinline__ void tc_fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Barrier among `count` threads (whole warps) of the CTA on hardware barrier
+// `id` (id 0 is the one __syncthreads uses).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------ tcgen05 MMA
 // D(tmem) (+)= A(smem) * B(smem), kind::f16 (bf16 in, fp32 accumulate).
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,

@@ -15,6 +15,15 @@ Workloads (the five shapes the method is measured on):
   page "Attention Is Memory-Bound, and Nobody Noticed for Five Years")
 * ``stress_65536_causal``    B=1,  H=32, N=65536, d=128, causal,     Q,K ~ N(0,4^2), V ~ U(-1,1)
 
+Inference shapes (Nq query rows against Nk keys, causal alignment bottom-right):
+
+* ``decode_131072``            B=4, H=32, Nq=1,   Nk=131072, d=128, Q,K,V ~ N(0,1)
+  (one new token per sequence against a 128K-token context, the upper end of
+  the 2K to 128K context growth on the pratikdhanave.com article "The
+  Attention Bottleneck - and How FlashAttention Fixed It", "Key takeaways")
+* ``chunk_128x32768_causal``   B=4, H=32, Nq=128, Nk=32768,  d=128, causal
+* ``chunk_512x8192_causal``    B=2, H=16, Nq=512, Nk=8192,   d=128, causal
+
 Draws are fp32 from a CPU ``torch.Generator`` seeded with the given seed, in the
 order Q, K, V, then rounded to bf16 (round to nearest even).
 """
@@ -58,6 +67,56 @@ WORKLOADS = {
         Workload("stress_65536_causal", 1, 32, 65536, 128, True, "stress", 1005, True),
     )
 }
+
+
+@dataclass(frozen=True)
+class KvWorkload:
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    dist: str
+    seed: int
+    rows_per_head: int  # query rows per (b, h) the parity check compares (all if >= Nq)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+KV_WORKLOADS = {
+    w.name: w
+    for w in (
+        KvWorkload("decode_131072", 4, 32, 1, 131072, 128, False, "normal", 1101, 1),
+        KvWorkload("chunk_128x32768_causal", 4, 32, 128, 32768, 128, True, "normal", 1102, 16),
+        KvWorkload("chunk_512x8192_causal", 2, 16, 512, 8192, 128, True, "normal", 1103, 32),
+    )
+}
+
+
+def _draw(g, shape, dist):
+    if dist == "normal":
+        return torch.randn(shape, generator=g, dtype=torch.float32)
+    if dist == "grid8":
+        return torch.randint(-32, 33, shape, generator=g).to(torch.float32) / 8.0
+    raise ValueError(f"unknown distribution {dist!r}")
+
+
+def make_q_kv(B: int, H: int, Nq: int, Nk: int, d: int, seed: int, dist: str = "normal"):
+    """Q [B, H, Nq, d] and K, V [B, H, Nk, d] as contiguous CPU bf16 tensors,
+    drawn in the order Q, K, V ("normal" or "grid8" as in make_qkv)."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    q = _draw(g, (B, H, Nq, d), dist)
+    k = _draw(g, (B, H, Nk, d), dist)
+    v = _draw(g, (B, H, Nk, d), dist)
+    return (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
+
+
+def make_kv_workload(w: KvWorkload):
+    return make_q_kv(w.B, w.H, w.Nq, w.Nk, w.d, w.seed, w.dist)
 
 
 def make_qkv(B: int, H: int, N: int, d: int, seed: int, dist: str = "normal"):

@@ -87,6 +87,60 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              attn_stream_t stream);
 
 /*
+ * attn_fwd_kv - fused attention of Nq query rows against Nk keys per head, the
+ * long-context inference shape (a few new tokens against a long context:
+ * pratikdhanave.com, "The Attention Bottleneck - and How FlashAttention Fixed
+ * It", "Key takeaways", on context grown from 2K to 128K tokens). The article
+ * describes no split of the key range; splitting it across CTAs and merging by
+ * log-sum-exp is this library's reading of how to keep every SM busy when
+ * B*H*ceil(Nq/128) CTAs cannot fill the GPU.
+ *
+ * q (in): [B, H, Nq, d] bf16. k, v (in): [B, H, Nk, d] bf16.
+ * o (out): [B, H, Nq, d] bf16. lse (out): [B, H, Nq] fp32.
+ * Causal alignment is bottom-right: query row i is sequence position
+ * i + (Nk - Nq), and sees key j iff j <= i + (Nk - Nq) (so Nq == Nk is the
+ * square causal problem of attn_fwd, and Nq = 1 sees every key). Causal needs
+ * Nq <= Nk (ATTN_ERR_SHAPE otherwise).
+ *
+ * The keys are cut into 128-key tiles and the tiles into num_splits ranges of
+ * equal length (the last may be shorter; a request above the tile count is
+ * clamped to it, and a count that would leave a range empty is lowered). Each
+ * (head, query block, range) is one CTA of the fused kernel, which writes a
+ * normalised fp32 partial O and its lse per range; a second kernel combines
+ * them, O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max_s lse_s).
+ * With num_splits = 1 the fused kernel writes o and lse directly.
+ *
+ * num_splits: 1 .. 256, or 0 for attn_fwd_kv_num_splits(...)'s choice.
+ * workspace: device memory of at least
+ * attn_fwd_kv_workspace_bytes(B, H, Nq, Nk, d, num_splits) bytes, 256-byte
+ * aligned; NULL is allowed when that is 0. Other conventions as for attn_fwd
+ * (B, H, Nq, Nk >= 1; B*H*Nq and B*H*Nk fit in a signed 32-bit int).
+ */
+int attn_fwd_kv(const void *q, const void *k, const void *v, void *o,
+                float *lse, int B, int H, int Nq, int Nk, int d, float scale,
+                int causal, int num_splits, void *workspace,
+                size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_fwd_kv_num_splits - the split count attn_fwd_kv uses for num_splits = 0
+ * on the current device: 1 when B*H*ceil(Nq/rows) CTAs already fill the SMs
+ * (rows = 128 for Nq <= 128, else 256), otherwise the fewest splits whose
+ * waves of CTAs are within 15% of the best SM utilisation, with at least 8 KV
+ * tiles per split. Returns a count >= 1, or a negative ATTN_ERR_* code.
+ */
+int attn_fwd_kv_num_splits(int B, int H, int Nq, int Nk, int d);
+
+/*
+ * attn_fwd_kv_workspace_bytes - workspace attn_fwd_kv needs for this shape and
+ * num_splits (0 = the automatic choice on the current device): with s > 1
+ * effective splits, s*B*H*Nq*d fp32 partial outputs (rounded up to 256 bytes)
+ * followed by s*B*H*Nq fp32 partial lse values; 0 when s = 1 or the arguments
+ * are invalid.
+ */
+size_t attn_fwd_kv_workspace_bytes(int B, int H, int Nq, int Nk, int d,
+                                   int num_splits);
+
+/*
  * attn_fwd_naive_workspace_bytes - bytes of workspace attn_fwd_naive needs:
  * 2 * (B*H*N*N) bf16 values (S, then P), i.e. 4*B*H*N*N bytes. Returns 0 if
  * the arguments are not positive or the size overflows.

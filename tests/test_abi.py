@@ -89,3 +89,39 @@ def test_product_path_has_no_fallback(monkeypatch):
     monkeypatch.setattr(ea, "_LIB_PATH", "/nonexistent/libattn_b200.so")
     with pytest.raises(RuntimeError):
         ea.lib()
+
+
+def _kv(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=2, Nq=1, Nk=1000, d=128, scale=0.125,
+                causal=0, splits=1, ws=None, ws_bytes=0, stream=None)
+    args.update(kw)
+    return ea.abi.attn_fwd_kv(args["q"], args["k"], args["v"], args["o"], args["lse"],
+                              args["B"], args["H"], args["Nq"], args["Nk"], args["d"],
+                              args["scale"], args["causal"], args["splits"], args["ws"],
+                              args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), -1), (dict(Nq=0), -2), (dict(Nk=0), -2), (dict(B=70000, H=70000), -2),
+    (dict(Nq=5, Nk=4, causal=1), -2),           # causal needs Nq <= Nk
+    (dict(d=80), -3), (dict(v=A + 4), -4), (dict(scale=0.0), -5), (dict(causal=3), -6),
+    (dict(splits=-1), -2), (dict(splits=257), -2),
+    (dict(splits=4), -1),                        # a split workspace is required
+    (dict(splits=4, ws=A + 16, ws_bytes=1 << 30), -4),   # 256-byte alignment
+    (dict(splits=4, ws=A, ws_bytes=100), -7),
+])
+def test_kv_argument_errors(L, kw, code):
+    assert _kv(**kw) == code
+
+
+def test_kv_workspace_bytes(L):
+    f = ea.abi.attn_fwd_kv_workspace_bytes
+    # 1000 keys = 8 tiles of 128; 4 splits of 2 tiles; [4][2][1][128] fp32 O + [4][2][1] lse
+    assert f(1, 2, 1, 1000, 128, 4) == 4 * 2 * 128 * 4 + 4 * 2 * 4 + (256 - (4 * 2 * 128 * 4) % 256) % 256
+    assert f(1, 2, 1, 1000, 128, 1) == 0
+    # more splits than tiles clamp to the tile count; 3 requested on 8 tiles -> 3 tiles per
+    # split -> 3 splits; 7 requested -> 2 tiles per split -> 4 splits (none empty)
+    assert f(1, 1, 3, 1000, 64, 100) == f(1, 1, 3, 1000, 64, 8)
+    assert f(1, 1, 3, 1000, 64, 7) == f(1, 1, 3, 1000, 64, 4)
+    assert f(1, 1, 3, 1000, 64, 3) == 3 * 3 * 64 * 4 + 3 * 3 * 4 + (256 - (3 * 3 * 64 * 4) % 256) % 256
+    assert f(0, 1, 3, 1000, 64, 3) == 0 and f(1, 1, 3, 1000, 96, 3) == 0
