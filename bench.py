@@ -52,6 +52,9 @@ def parse_args(argv=None):
     p.add_argument("--workload", default=WORKLOAD)
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-naive", action="store_true", help="skip the unfused traffic line")
+    p.add_argument("--no-kv", action="store_true", help="skip the split-KV inference lines")
+    p.add_argument("--kv-only", default=None, metavar="WORKLOAD",
+                   help="run only the split-KV line of this inference workload (one GPU)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU time of the oracle sample")
@@ -277,6 +280,13 @@ def run_ours(args):
     from exact_attention_125_b200.inputs import WORKLOADS, make_workload
 
     world, rank, local = dist_env()
+    if args.kv_only:
+        torch.cuda.set_device(local)
+        peaks, _ = load_peaks()
+        line = split_kv_line(args.kv_only, torch.device("cuda", local), peaks,
+                             steps=args.steps, warmup=args.warmup)
+        print(json.dumps({"split_kv": line}), flush=True)
+        return 0
     if world != args.gpus:
         if not (world == 1 and args.gpus == 1):
             raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch with torchrun")
@@ -325,6 +335,8 @@ def run_ours(args):
     e2e = (e2e_through_abi(args, w, qh, kh, vh, device, dist, flops, world)
            if args.e2e_steps > 0 else None)
     naive = None if args.no_naive else naive_line(w, device, peaks)
+    split_kv = None if args.no_kv else [split_kv_line(name, device, peaks)
+                                       for name in KV_BENCH_WORKLOADS]
 
     peak = float(peaks["bf16_tflops"])
     line = {
@@ -367,6 +379,8 @@ def run_ours(args):
     }
     if naive is not None:
         line["naive"] = naive
+    if split_kv is not None:
+        line["split_kv"] = split_kv
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, n, cores, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -471,6 +485,61 @@ def naive_line(w, device, peaks, steps=2):
             "hbm_peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
             "tflops": costs.attn_flops(w.B, w.H, w.N, w.d, w.causal) / (ms * 1e-3) / 1e12,
             "head_group": group, "launches_per_step": 3 * (BH // group)}
+
+
+KV_BENCH_WORKLOADS = ("decode_131072", "chunk_128x32768_causal")
+
+
+def split_kv_line(name, device, peaks, steps=10, warmup=3):
+    """attn_fwd_kv on an inference workload with the library's automatic split
+    count (inputs larger than L2); reported as achieved HBM GB/s of its
+    algorithmic traffic (Q, K, V read once, O and lse written once) and as
+    TFLOP/s of the visible (query, key) pairs."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    from exact_attention_125_b200 import costs
+    from exact_attention_125_b200.inputs import KV_WORKLOADS
+    w = KV_WORKLOADS[name]
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    q = torch.randn((w.B, w.H, w.Nq, w.d), device=device, generator=g).to(torch.bfloat16)
+    k = torch.randn((w.B, w.H, w.Nk, w.d), device=device, generator=g).to(torch.bfloat16)
+    v = torch.randn((w.B, w.H, w.Nk, w.d), device=device, generator=g).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=device)
+    splits = ea.kv_num_splits(w.B, w.H, w.Nq, w.Nk, w.d)
+    ws_bytes = ea.kv_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d, splits)
+    ws = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        ea.attn_fwd_kv(q, k, v, o, lse, scale=w.scale, causal=w.causal, num_splits=splits,
+                       workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    if ea.last_device_error() != 0:
+        raise SystemExit(f"device watchdog fired in the split-KV line {name}")
+    ms = start.elapsed_time(end) / steps
+    nbytes = costs.kv_bytes(w.B, w.H, w.Nq, w.Nk, w.d)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    flops = costs.kv_flops(w.B, w.H, w.Nq, w.Nk, w.d, w.causal)
+    del q, k, v, ws
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+            "causal": w.causal, "num_splits": splits, "ms_per_step": ms, "steps": steps,
+            "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+            "hbm_peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
+            "bound": "hbm", "tflops": flops / (ms * 1e-3) / 1e12,
+            "launches_per_step": 2 if splits > 1 else 1,
+            "l2": "inputs larger than L2"}
 
 
 def main(argv=None):

@@ -11,6 +11,11 @@
   P read) as traced on the anylearn.cc page "Attention Is Memory-Bound, and
   Nobody Noticed for Five Years"; on top of that Q, K, V are read and O and
   the log-sum-exp are written once.
+* Inference shapes (Nq query rows against Nk keys, causal alignment
+  bottom-right): query i sees min(Nk, i + Nk - Nq + 1) keys when causal, all
+  Nk otherwise; FLOPs are 4*d per (query, visible key) pair. The fused kernel
+  reads Q, K, V once and writes O and lse once: 2*B*H*(2*Nq + 2*Nk)*d + 4*B*H*Nq
+  bytes (the split partials and their combine are overhead, not algorithmic).
 """
 from __future__ import annotations
 
@@ -57,3 +62,21 @@ def tile_pairs(B: int, H: int, N: int, causal: bool, tile: int = 128) -> int:
     t = -(-N // tile)
     per_head = t * (t + 1) // 2 if causal else t * t
     return B * H * per_head
+
+
+def kv_visible_pairs(Nq: int, Nk: int, causal: bool) -> int:
+    """(query, key) pairs with the key visible, per head."""
+    if not causal:
+        return Nq * Nk
+    if Nq > Nk:
+        raise ValueError("causal needs Nq <= Nk")
+    # query i sees i + (Nk - Nq) + 1 <= Nk keys
+    return Nq * (Nk - Nq + 1) + Nq * (Nq - 1) // 2
+
+
+def kv_flops(B: int, H: int, Nq: int, Nk: int, d: int, causal: bool) -> float:
+    return 4.0 * B * H * d * kv_visible_pairs(Nq, Nk, causal)
+
+
+def kv_bytes(B: int, H: int, Nq: int, Nk: int, d: int) -> int:
+    return 2 * B * H * (2 * Nq + 2 * Nk) * d + 4 * B * H * Nq

@@ -21,6 +21,8 @@ Inference shapes (Nq query rows against Nk keys, causal alignment bottom-right):
   (one new token per sequence against a 128K-token context, the upper end of
   the 2K to 128K context growth on the pratikdhanave.com article "The
   Attention Bottleneck - and How FlashAttention Fixed It", "Key takeaways")
+* ``decode_32768``             B=4, H=32, Nq=1,   Nk=32768,  d=128 (the same at a
+  quarter of the context: small enough for multi-pass profiler captures)
 * ``chunk_128x32768_causal``   B=4, H=32, Nq=128, Nk=32768,  d=128, causal
 * ``chunk_512x8192_causal``    B=2, H=16, Nq=512, Nk=8192,   d=128, causal
 
@@ -91,6 +93,7 @@ KV_WORKLOADS = {
     w.name: w
     for w in (
         KvWorkload("decode_131072", 4, 32, 1, 131072, 128, False, "normal", 1101, 1),
+        KvWorkload("decode_32768", 4, 32, 1, 32768, 128, False, "normal", 1104, 1),
         KvWorkload("chunk_128x32768_causal", 4, 32, 128, 32768, 128, True, "normal", 1102, 16),
         KvWorkload("chunk_512x8192_causal", 2, 16, 512, 8192, 128, True, "normal", 1103, 32),
     )

@@ -121,3 +121,26 @@ def test_workload_table():
     w = WORKLOADS["long_8192_causal"]
     assert (w.B, w.H, w.N, w.d, w.causal) == (8, 32, 8192, 128, True)
     assert [x.seed for x in WORKLOADS.values()] == [1001, 1002, 1003, 1004, 1005]
+
+
+@pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 9), (3, 10), (5, 5), (17, 300)])
+def test_kv_visible_pairs_count_the_mask(Nq, Nk):
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    assert costs.kv_visible_pairs(Nq, Nk, True) == int((j <= i + (Nk - Nq)).sum())
+    assert costs.kv_visible_pairs(Nq, Nk, False) == Nq * Nk
+    assert costs.kv_flops(2, 3, Nq, Nk, 64, True) == 4.0 * 2 * 3 * 64 * int((j <= i + (Nk - Nq)).sum())
+
+
+def test_kv_bytes_decode_example():
+    # one query row against 131072 keys, d = 128, 4 x 32 heads: K and V dominate
+    b = costs.kv_bytes(4, 32, 1, 131072, 128)
+    assert b == 128 * (2 * 128 * 2 + 2 * 131072 * 128 * 2 + 4)
+
+
+def test_kv_inputs_shapes_and_determinism():
+    from exact_attention_125_b200.inputs import make_q_kv
+    q, k, v = make_q_kv(1, 2, 3, 7, 8, seed=5)
+    assert q.shape == (1, 2, 3, 8) and k.shape == v.shape == (1, 2, 7, 8)
+    q2, k2, v2 = make_q_kv(1, 2, 3, 7, 8, seed=5)
+    assert torch.equal(q, q2) and torch.equal(k, k2) and torch.equal(v, v2)
