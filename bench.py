@@ -36,6 +36,7 @@ if ROOT not in sys.path:
 WORKLOAD = "long_8192_causal"
 METRIC = "attn fwd TFLOP/s (causal-adjusted) and % of B200 dense BF16 peak"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_attn_fwd_long_8192_causal.txt")
+KV_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_attn_fwd_kv_decode.txt")
 # the sources that define the fused kernel; the ncu summary records their hash
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_125_b200", "csrc", f)
                   for f in ("fused_fwd.cu", "sm100.cuh", "tmem_io.cuh", "watchdog.cuh",
@@ -78,22 +79,47 @@ def source_hash(paths=None) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    or None when the summary is missing or was taken on another kernel source."""
-    if not os.path.exists(PROFILE_SUMMARY):
+def _summary_fields(path):
+    """key: value lines of a committed ncu summary, or None when it is missing
+    or was taken on another kernel source."""
+    if not os.path.exists(path):
         return None
     fields = {}
-    for line in open(PROFILE_SUMMARY):
+    for line in open(path):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             fields[k.strip()] = v.strip()
     if fields.get("kernel_source_sha256_16") != source_hash():
         return None
+    return fields
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary."""
+    fields = _summary_fields(PROFILE_SUMMARY)
     try:
-        return float(fields["dram_bytes_per_launch_full_workload"])
+        return float(fields["dram_bytes_per_launch_full_workload"]) if fields else None
     except (KeyError, ValueError):
         return None
+
+
+def profiled_kv_traffic(w):
+    """DRAM bytes per launch of the split-KV kernel on a decode workload: the
+    capture's reads scaled by the key count (every K/V byte is read once, so
+    reads grow with Nk), plus its writes. None for other shapes."""
+    fields = _summary_fields(KV_PROFILE_SUMMARY)
+    if not fields or w.Nq != 1 or w.causal:
+        return None
+    from exact_attention_125_b200.inputs import KV_WORKLOADS
+    base = KV_WORKLOADS.get(fields.get("workload", ""))
+    if base is None or (base.B, base.H, base.Nq, base.d) != (w.B, w.H, w.Nq, w.d):
+        return None
+    try:
+        reads = float(fields["dram_bytes_read_per_launch"])
+        writes = float(fields["dram_bytes_write_per_launch"])
+    except (KeyError, ValueError):
+        return None
+    return reads * w.Nk / base.Nk + writes
 
 
 # ------------------------------------------------------------------ clocks
@@ -371,7 +397,7 @@ def run_ours(args):
             "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peaks_kind}, burst)",
             "traffic": profiled_traffic(),
             "algorithmic_bytes": costs.fused_bytes(w.B, w.H, w.N, w.d),
-            "kernel": "fused_attn_fwd_kernel<128>",
+            "kernel": "fused_attn_fwd_kernel<128, false>",
         },
         "clocks": {k: clock_info[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "e2e": e2e,
@@ -537,7 +563,10 @@ def split_kv_line(name, device, peaks, steps=10, warmup=3):
             "causal": w.causal, "num_splits": splits, "ms_per_step": ms, "steps": steps,
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
-            "bound": "hbm", "tflops": flops / (ms * 1e-3) / 1e12,
+            "bound": "hbm", "traffic": profiled_kv_traffic(w),
+            "kernel": "fused_attn_fwd_kernel<128, true>" + (" + lse_combine_kernel<128>"
+                                                            if splits > 1 else ""),
+            "tflops": flops / (ms * 1e-3) / 1e12,
             "launches_per_step": 2 if splits > 1 else 1,
             "l2": "inputs larger than L2"}
 

@@ -13,12 +13,20 @@
 // 128-row query tiles "a" and "b" that ping-pong: while the softmax warps of
 // one tile turn S into P, the tensor core runs the other tile's MMAs.
 //
-// Roles (320 threads):
+// Roles (384 threads):
 //   warps 0-3  softmax + epilogue of query tile a (thread t owns row t)
 //   warps 4-7  softmax + epilogue of query tile b
 //   warp  8    TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... into
 //              a ring of shared-memory stages (128B-swizzled, mbarrier-tracked)
 //   warp  9    tensor-memory allocator and single-thread tcgen05 MMA issuer
+//   warps 10-11 only hand their registers to the softmax warps (setmaxnreg)
+//
+// The kv instantiation (kKV = true) serves Nq query rows against N keys with
+// the keys of each head cut into ranges that separate CTAs attend to: a CTA is
+// (head, key range, query block); with Nq <= 128 its one query tile is shared
+// by both softmax warpgroups, which take alternate KV tiles and merge their
+// (O, m, l) at the end. Several ranges leave fp32 partial (O, lse) pairs that
+// lse_combine_kernel (combine.cu) merges.
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_a [0,128), S_b [128,256),
 // O_a [256, 256+d), O_b [256+d, 256+2d). P (bf16, two per column) overwrites
