@@ -63,6 +63,13 @@ def _load():
                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                            ctypes.c_double, ctypes.c_int, i64p, ctypes.c_int64, f64p, f64p,
                            ctypes.c_int]
+        for name in ("oracle_attn_ext_bf16", "oracle_attn_ext_f64"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_void_p, i64p, ctypes.c_int64, f64p, f64p, ctypes.c_int]
         lib.oracle_probs_f64.restype = ctypes.c_int
         lib.oracle_probs_f64.argtypes = [f64p, f64p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_double, ctypes.c_int,
@@ -151,6 +158,46 @@ def attention_kv(q, k, v, scale: float, causal: bool, rows=None, nthreads: int =
     lse = np.zeros((R,), dtype=np.float64)
     st = fn(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, B, H, Nq, Nk, d, float(scale),
             int(bool(causal)), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
+            o.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+            lse.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), int(nthreads))
+    if st != 0:
+        raise RuntimeError(f"oracle failed with status {st}")
+    return o, lse
+
+
+def attention_ext(q, k, v, scale: float, causal: bool, window_left: int = -1,
+                  window_right: int = -1, slopes=None, rows=None, nthreads: int = 0):
+    """attention_kv with a key window and a linear distance bias. Query i is
+    sequence position pos = i + Nk - Nq; key j is allowed iff j <= pos when
+    causal, pos - window_left <= j when window_left >= 0 and j <= pos +
+    window_right when window_right >= 0; with slopes (H values) the score of
+    key j is lowered by slopes[h] * |pos - j|. Returns (o, lse)."""
+    lib = _load()
+    if isinstance(q, np.ndarray):
+        qa, ka, va = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+        fn = lib.oracle_attn_ext_f64
+    else:
+        qa, ka, va = (_as_bf16_bits(x) for x in (q, k, v))
+        fn = lib.oracle_attn_ext_bf16
+    if qa.ndim != 4 or ka.shape != va.shape or ka.shape[:2] != qa.shape[:2] or ka.shape[3] != qa.shape[3]:
+        raise ValueError("q [B, H, Nq, d] and k, v [B, H, Nk, d] expected")
+    B, H, Nq, d = (int(x) for x in qa.shape)
+    Nk = int(ka.shape[2])
+    sl = None
+    if slopes is not None:
+        sl = np.ascontiguousarray(np.asarray(slopes, dtype=np.float64).reshape(-1))
+        if sl.shape[0] != H:
+            raise ValueError("one slope per head expected")
+    if rows is None:
+        rows = all_rows(B * H, Nq)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+    R = rows.shape[0]
+    o = np.zeros((R, d), dtype=np.float64)
+    lse = np.zeros((R,), dtype=np.float64)
+    st = fn(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, B, H, Nq, Nk, d, float(scale),
+            int(bool(causal)), int(window_left), int(window_right),
+            sl.ctypes.data if sl is not None else None,
+            rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
             o.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
             lse.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), int(nthreads))
     if st != 0:

@@ -62,13 +62,16 @@ static double load_elem(const void *base, int kind, int64_t idx) {
     return bf16_bits_to_double(((const uint16_t *)base)[idx]);
 }
 
-/* Step 1: the row of scores for query q (length d) against keys 0..nkeys-1. */
-static void scores_row(const double *q, const double *K, int nkeys, int d,
-                       double scale, double *s) {
-    for (int j = 0; j < nkeys; ++j) {
+/* Step 1: the scores of query q (length d, sequence position pos) against
+ * keys j0..j1-1: s[j - j0] = scale * q.K[j] - slope * |pos - j| (the second
+ * term is the linear distance bias; slope = 0 leaves the plain score). */
+static void scores_row(const double *q, const double *K, int j0, int j1, int d,
+                       double scale, double slope, int64_t pos, double *s) {
+    for (int j = j0; j < j1; ++j) {
         double dot = 0.0;
         for (int c = 0; c < d; ++c) dot += q[c] * K[(int64_t)j * d + c];
-        s[j] = scale * dot;
+        s[j - j0] = scale * dot;
+        if (slope != 0.0) s[j - j0] -= slope * fabs((double)(pos - j));
     }
 }
 
@@ -87,36 +90,47 @@ static void softmax_row(double *s, int n, double *m_out, double *l_out) {
     *l_out = l;
 }
 
-/* Step 3: o = sum_j p_j * V[j,:]. */
-static void output_row(const double *p, const double *V, int n, int d, double *o) {
+/* Step 3: o = sum_j p_j * V[j,:] over keys j0..j1-1 (p indexed from j0). */
+static void output_row(const double *p, const double *V, int j0, int j1, int d,
+                       double *o) {
     for (int c = 0; c < d; ++c) o[c] = 0.0;
-    for (int j = 0; j < n; ++j)
-        for (int c = 0; c < d; ++c) o[c] += p[j] * V[(int64_t)j * d + c];
+    for (int j = j0; j < j1; ++j)
+        for (int c = 0; c < d; ++c) o[c] += p[j - j0] * V[(int64_t)j * d + c];
 }
 
-/* One query row of one head: steps 1-3 and the log-sum-exp. nkeys is the
- * number of allowed keys (a prefix of the head's keys). */
-static void attend_row(const double *q, const double *K, const double *V, int nkeys,
-                       int d, double scale, double *s_buf, double *o, double *lse) {
-    if (nkeys <= 0) {
+/* One query row of one head: steps 1-3 and the log-sum-exp over the allowed
+ * keys j0..j1-1. */
+static void attend_row(const double *q, const double *K, const double *V, int j0,
+                       int j1, int d, double scale, double slope, int64_t pos,
+                       double *s_buf, double *o, double *lse) {
+    if (j1 <= j0) {
         for (int c = 0; c < d; ++c) o[c] = 0.0;
         *lse = -INFINITY;
         return;
     }
     double m, l;
-    scores_row(q, K, nkeys, d, scale, s_buf);
-    softmax_row(s_buf, nkeys, &m, &l);
-    output_row(s_buf, V, nkeys, d, o);
+    scores_row(q, K, j0, j1, d, scale, slope, pos, s_buf);
+    softmax_row(s_buf, j1 - j0, &m, &l);
+    output_row(s_buf, V, j0, j1, d, o);
     *lse = m + log(l);
 }
 
-/* Allowed keys of query i: all Nk, or those j <= i + (Nk - Nq) when causal. */
-static int allowed_keys(int i, int Nq, int Nk, int causal) {
-    if (!causal) return Nk;
-    long long n = (long long)i + (Nk - Nq) + 1;
-    if (n > Nk) n = Nk;
-    if (n < 0) n = 0;
-    return (int)n;
+/* Allowed keys of query i, as the range j0..j1-1. Query i is sequence
+ * position pos = i + (Nk - Nq). Key j is allowed iff j < Nk, and j <= pos when
+ * causal, and j >= pos - wl when wl >= 0, and j <= pos + wr when wr >= 0
+ * (a window of wl keys before the query's position and wr after it; a
+ * negative bound means unbounded on that side). */
+static void key_range(int i, int Nq, int Nk, int causal, int wl, int wr, int *j0,
+                      int *j1) {
+    int64_t pos = (int64_t)i + (Nk - Nq);
+    int64_t hi = Nk - 1;
+    if (causal && pos < hi) hi = pos;
+    if (wr >= 0 && pos + wr < hi) hi = pos + wr;
+    int64_t lo = 0;
+    if (wl >= 0 && pos - wl > lo) lo = pos - wl;
+    if (hi < lo - 1) hi = lo - 1;
+    *j0 = (int)lo;
+    *j1 = (int)(hi + 1);
 }
 
 typedef struct {
@@ -130,6 +144,8 @@ typedef struct {
     const int64_t *mine;  /* indices into rows[] for this head */
     int64_t nmine;
     int Nq;               /* query rows per head (N is the key count) */
+    int wl, wr;           /* window bounds, negative = unbounded */
+    double slope;         /* distance-bias slope of this head (0 = none) */
     int tid, nthreads;
     double *o, *lse;
     int ok;        /* set to 1 by run_job when its rows are done */
@@ -151,8 +167,11 @@ static void *run_job(void *arg) {
         int i = (int)jb->rows[2 * r + 1];
         int64_t qoff = (jb->bh * jb->Nq + i) * (int64_t)jb->d;
         for (int c = 0; c < jb->d; ++c) qrow[c] = load_elem(jb->q, jb->kind, qoff + c);
-        attend_row(qrow, jb->K, jb->V, allowed_keys(i, jb->Nq, jb->N, jb->causal), jb->d,
-                   jb->scale, s, jb->o + r * (int64_t)jb->d, jb->lse + r);
+        int j0, j1;
+        key_range(i, jb->Nq, jb->N, jb->causal, jb->wl, jb->wr, &j0, &j1);
+        attend_row(qrow, jb->K, jb->V, j0, j1, jb->d, jb->scale, jb->slope,
+                   (int64_t)i + (jb->N - jb->Nq), s, jb->o + r * (int64_t)jb->d,
+                   jb->lse + r);
     }
     free(s);
     free(qrow);
@@ -166,13 +185,16 @@ int oracle_default_threads(void) {
 }
 
 static int attend(const void *q, const void *k, const void *v, int kind, int B,
-                  int H, int Nq, int N, int d, double scale, int causal,
-                  const int64_t *rows, int64_t nrows, double *o, double *lse,
-                  int nthreads) {
+                  int H, int Nq, int N, int d, double scale, int causal, int wl,
+                  int wr, const double *slopes, const int64_t *rows, int64_t nrows,
+                  double *o, double *lse, int nthreads) {
     if (!q || !k || !v || !rows || !o || !lse) return -1;
     if (B <= 0 || H <= 0 || Nq <= 0 || N <= 0 || d <= 0 || nrows < 0) return -2;
     if (causal && Nq > N) return -2;
     if (!isfinite(scale)) return -3;
+    if (slopes)
+        for (int h = 0; h < H; ++h)
+            if (!isfinite(slopes[h])) return -3;
     if (nthreads <= 0) nthreads = oracle_default_threads();
     int64_t BH = (int64_t)B * H;
     for (int64_t r = 0; r < nrows; ++r) {
@@ -200,8 +222,9 @@ static int attend(const void *q, const void *k, const void *v, int kind, int B,
         }
         int nt = nmine < nthreads ? (int)nmine : nthreads;
         for (int t = 0; t < nt; ++t) {
+            double slope = slopes ? slopes[bh % H] : 0.0;
             job_t jb = {q, kind, K, V, bh, N, d, causal, scale, rows, mine, nmine, Nq,
-                        t, nt, o, lse, 0, 0};
+                        wl, wr, slope, t, nt, o, lse, 0, 0};
             jobs[t] = jb;
         }
         /* A thread that cannot be created runs its share inline. */
@@ -232,8 +255,8 @@ int oracle_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      int B, int H, int N, int d, double scale, int causal,
                      const int64_t *rows, int64_t nrows, double *o, double *lse,
                      int nthreads) {
-    return attend(q, k, v, IN_BF16, B, H, N, N, d, scale, causal, rows, nrows, o,
-                  lse, nthreads);
+    return attend(q, k, v, IN_BF16, B, H, N, N, d, scale, causal, -1, -1, NULL, rows,
+                  nrows, o, lse, nthreads);
 }
 
 /* Same as oracle_attn_bf16 with double inputs (values need not be bf16). */
@@ -241,8 +264,8 @@ int oracle_attn_f64(const double *q, const double *k, const double *v, int B,
                     int H, int N, int d, double scale, int causal,
                     const int64_t *rows, int64_t nrows, double *o, double *lse,
                     int nthreads) {
-    return attend(q, k, v, IN_F64, B, H, N, N, d, scale, causal, rows, nrows, o,
-                  lse, nthreads);
+    return attend(q, k, v, IN_F64, B, H, N, N, d, scale, causal, -1, -1, NULL, rows,
+                  nrows, o, lse, nthreads);
 }
 
 /* Nq queries against Nk keys per head: q is [B, H, Nq, d], k and v are
@@ -252,8 +275,8 @@ int oracle_attn_kv_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int B, int H, int Nq, int Nk, int d, double scale,
                         int causal, const int64_t *rows, int64_t nrows, double *o,
                         double *lse, int nthreads) {
-    return attend(q, k, v, IN_BF16, B, H, Nq, Nk, d, scale, causal, rows, nrows, o,
-                  lse, nthreads);
+    return attend(q, k, v, IN_BF16, B, H, Nq, Nk, d, scale, causal, -1, -1, NULL, rows,
+                  nrows, o, lse, nthreads);
 }
 
 /* Same with double inputs. */
@@ -261,8 +284,33 @@ int oracle_attn_kv_f64(const double *q, const double *k, const double *v, int B,
                        int H, int Nq, int Nk, int d, double scale, int causal,
                        const int64_t *rows, int64_t nrows, double *o, double *lse,
                        int nthreads) {
-    return attend(q, k, v, IN_F64, B, H, Nq, Nk, d, scale, causal, rows, nrows, o,
-                  lse, nthreads);
+    return attend(q, k, v, IN_F64, B, H, Nq, Nk, d, scale, causal, -1, -1, NULL, rows,
+                  nrows, o, lse, nthreads);
+}
+
+/* Masked and position-biased variants (the "custom attention bias, unusual
+ * masking pattern, novel position encoding" cases that the anylearn.cc page
+ * says fall off a fused library's fast path): keys limited to the window
+ * [pos - wl, pos + wr] (negative bound = unbounded) on top of the causal
+ * rule, and, when slopes is not NULL, the score of key j for a query at
+ * position pos lowered by slopes[h] * |pos - j| (a linear distance bias per
+ * head h). wl = wr = -1 with slopes = NULL is oracle_attn_kv_*. */
+int oracle_attn_ext_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         int B, int H, int Nq, int Nk, int d, double scale,
+                         int causal, int wl, int wr, const double *slopes,
+                         const int64_t *rows, int64_t nrows, double *o, double *lse,
+                         int nthreads) {
+    return attend(q, k, v, IN_BF16, B, H, Nq, Nk, d, scale, causal, wl, wr, slopes,
+                  rows, nrows, o, lse, nthreads);
+}
+
+/* Same with double inputs. */
+int oracle_attn_ext_f64(const double *q, const double *k, const double *v, int B,
+                        int H, int Nq, int Nk, int d, double scale, int causal, int wl,
+                        int wr, const double *slopes, const int64_t *rows,
+                        int64_t nrows, double *o, double *lse, int nthreads) {
+    return attend(q, k, v, IN_F64, B, H, Nq, Nk, d, scale, causal, wl, wr, slopes, rows,
+                  nrows, o, lse, nthreads);
 }
 
 /* The probability row p[0..N-1] of query i for a single head (q: [N, d],
@@ -270,10 +318,11 @@ int oracle_attn_kv_f64(const double *q, const double *k, const double *v, int B,
 int oracle_probs_f64(const double *q, const double *k, int N, int d,
                      double scale, int causal, int i, double *p) {
     if (!q || !k || !p || N <= 0 || d <= 0 || i < 0 || i >= N) return -1;
-    int nkeys = allowed_keys(i, N, N, causal);
+    int j0, j1;
+    key_range(i, N, N, causal, -1, -1, &j0, &j1);
     double m, l;
     for (int j = 0; j < N; ++j) p[j] = 0.0;
-    scores_row(q + (int64_t)i * d, k, nkeys, d, scale, p);
-    softmax_row(p, nkeys, &m, &l);
+    scores_row(q + (int64_t)i * d, k, j0, j1, d, scale, 0.0, i, p + j0);
+    softmax_row(p + j0, j1 - j0, &m, &l);
     return 0;
 }

@@ -253,3 +253,81 @@ def test_kv_single_query_causal_sees_every_key():
     o_c, l_c = oracle.attention_kv(q, k, v, 0.5, True)
     o_n, l_n = oracle.attention_kv(q, k, v, 0.5, False)
     assert np.array_equal(o_c, o_n) and np.array_equal(l_c, l_n)
+
+
+# ------------------------------------------------ key windows, distance bias
+def _ext_brute(q, k, v, scale, causal, wl, wr, slopes):
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    logits = torch.einsum("bhid,bhjd->bhij", tq, tk) * scale
+    pos = torch.arange(Nq)[:, None] + (Nk - Nq)
+    j = torch.arange(Nk)[None, :]
+    if slopes is not None:
+        logits = logits - torch.tensor(slopes, dtype=torch.float64)[None, :, None, None] * \
+            (pos - j).abs().to(torch.float64)
+    allowed = torch.ones(Nq, Nk, dtype=torch.bool)
+    if causal:
+        allowed &= j <= pos
+    if wl >= 0:
+        allowed &= j >= pos - wl
+    if wr >= 0:
+        allowed &= j <= pos + wr
+    logits = logits.masked_fill(~allowed, float("-inf"))
+    return torch.softmax(logits, -1) @ tv, torch.logsumexp(logits, -1)
+
+
+@pytest.mark.parametrize("causal,wl,wr,alibi", [
+    (True, 3, -1, False), (False, 2, 1, False), (False, -1, 0, False), (False, 4, -1, True),
+    (True, -1, -1, True), (True, 5, -1, True), (False, 0, 0, False), (False, 2, 3, True),
+])
+@pytest.mark.parametrize("Nq,Nk", [(1, 9), (6, 6), (4, 13)])
+def test_ext_brute_force(Nq, Nk, causal, wl, wr, alibi):
+    B, H, d = 2, 3, 4
+    q = RNG.standard_normal((B, H, Nq, d))
+    k = RNG.standard_normal((B, H, Nk, d))
+    v = RNG.standard_normal((B, H, Nk, d))
+    slopes = [0.5, 0.25, 0.125] if alibi else None
+    o, lse = oracle.attention_ext(q, k, v, 0.4, causal, wl, wr, slopes)
+    o_ref, lse_ref = _ext_brute(q, k, v, 0.4, causal, wl, wr, slopes)
+    assert np.abs(o - o_ref.numpy().reshape(-1, d)).max() <= 1e-12
+    assert np.abs(lse - lse_ref.numpy().reshape(-1)).max() <= 1e-12
+
+
+def test_ext_without_options_is_attention_kv():
+    q = RNG.standard_normal((1, 2, 5, 8))
+    k = RNG.standard_normal((1, 2, 20, 8))
+    v = RNG.standard_normal((1, 2, 20, 8))
+    for causal in (False, True):
+        o1, l1 = oracle.attention_kv(q, k, v, 0.3, causal)
+        o2, l2 = oracle.attention_ext(q, k, v, 0.3, causal, -1, -1, None)
+        o3, l3 = oracle.attention_ext(q, k, v, 0.3, causal, 100, 100, [0.0, 0.0])  # window covers all
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+        assert np.array_equal(o1, o3) and np.array_equal(l1, l3)
+
+
+def test_ext_diagonal_window_and_steep_bias_pick_the_own_position():
+    # a window of width 0 leaves the query's own position: o = v[pos],
+    # lse = scale q.k[pos]; a steep distance bias converges to the same o
+    Nq, Nk, d = 4, 10, 6
+    q = RNG.standard_normal((1, 1, Nq, d))
+    k = RNG.standard_normal((1, 1, Nk, d))
+    v = RNG.standard_normal((1, 1, Nk, d))
+    pos = np.arange(Nq) + Nk - Nq
+    o, lse = oracle.attention_ext(q, k, v, 0.5, False, 0, 0, None)
+    assert np.array_equal(o, v[0, 0, pos])
+    assert np.allclose(lse, 0.5 * np.einsum("id,id->i", q[0, 0], k[0, 0, pos]), rtol=0, atol=1e-15)
+    # slope 60: the next key's weight is below exp(-60 + |logit differences|) ~ 1e-22
+    o2, _ = oracle.attention_ext(q, k, v, 0.5, True, -1, -1, [60.0])
+    assert np.abs(o2 - v[0, 0, pos]).max() <= 1e-15
+
+
+def test_ext_bias_vanishes_at_the_own_position():
+    # with a causal window of width 0 the only allowed key is the query's own
+    # position, where the distance bias is slope * 0 = 0: nothing changes
+    q = RNG.standard_normal((1, 1, 3, 4))
+    k = RNG.standard_normal((1, 1, 7, 4))
+    v = RNG.standard_normal((1, 1, 7, 4))
+    o1, l1 = oracle.attention_ext(q, k, v, 0.5, True, 0, -1, None)
+    o2, l2 = oracle.attention_ext(q, k, v, 0.5, True, 0, -1, [3.0])
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)  # |pos - pos| = 0
