@@ -54,6 +54,7 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-naive", action="store_true", help="skip the unfused traffic line")
     p.add_argument("--no-kv", action="store_true", help="skip the split-KV inference lines")
+    p.add_argument("--no-ext", action="store_true", help="skip the window / distance-bias lines")
     p.add_argument("--kv-only", default=None, metavar="WORKLOAD",
                    help="run only the split-KV line of this inference workload (one GPU)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -363,6 +364,7 @@ def run_ours(args):
     naive = None if args.no_naive else naive_line(w, device, peaks)
     split_kv = None if args.no_kv else [split_kv_line(name, device, peaks)
                                        for name in KV_BENCH_WORKLOADS]
+    ext = None if args.no_ext else [ext_line(spec, device, peaks) for spec in EXT_BENCH]
 
     peak = float(peaks["bf16_tflops"])
     line = {
@@ -407,6 +409,8 @@ def run_ours(args):
         line["naive"] = naive
     if split_kv is not None:
         line["split_kv"] = split_kv
+    if ext is not None:
+        line["masks_and_bias"] = ext
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, n, cores, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -569,6 +573,62 @@ def split_kv_line(name, device, peaks, steps=10, warmup=3):
             "tflops": flops / (ms * 1e-3) / 1e12,
             "launches_per_step": 2 if splits > 1 else 1,
             "l2": "inputs larger than L2"}
+
+
+# (name, B, H, Nq, Nk, d, causal, window_left, window_right, distance bias)
+EXT_BENCH = (
+    ("window_4096_of_32768_causal", 2, 32, 32768, 32768, 128, True, 4095, -1, False),
+    ("alibi_8192_causal", 8, 32, 8192, 8192, 128, True, -1, -1, True),
+)
+
+
+def ext_line(spec, device, peaks, steps=5, warmup=3):
+    """attn_fwd_ext on a sliding-window or distance-biased shape: TFLOP/s of
+    the allowed (query, key) pairs (4 d FLOP each) against the tensor peak."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    from exact_attention_125_b200 import costs
+    name, B, H, Nq, Nk, d, causal, wl, wr, bias = spec
+    g = torch.Generator(device=device).manual_seed(4242)
+    q = torch.randn((B, H, Nq, d), device=device, generator=g).to(torch.bfloat16)
+    k = torch.randn((B, H, Nk, d), device=device, generator=g).to(torch.bfloat16)
+    v = torch.randn((B, H, Nk, d), device=device, generator=g).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=device)
+    slopes = (torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32,
+                           device=device) if bias else None)
+    splits = ea.ext_num_splits(B, H, Nq, Nk, d, wl)
+    ws_bytes = ea.ext_workspace_bytes(B, H, Nq, Nk, d, wl, splits)
+    ws = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        ea.attn_fwd_ext(q, k, v, o, lse, scale=1.0 / math.sqrt(d), causal=causal, window_left=wl,
+                        window_right=wr, alibi_slopes=slopes, num_splits=splits, workspace=ws,
+                        stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    if ea.last_device_error() != 0:
+        raise SystemExit(f"device watchdog fired in the line {name}")
+    ms = start.elapsed_time(end) / steps
+    flops = 4.0 * B * H * d * costs.ext_visible_pairs(Nq, Nk, causal, wl, wr)
+    tf = flops / (ms * 1e-3) / 1e12
+    del q, k, v, ws
+    torch.cuda.empty_cache()
+    return {"workload": name, "B": B, "H": H, "Nq": Nq, "Nk": Nk, "d": d, "causal": causal,
+            "window_left": wl, "window_right": wr, "distance_bias": bias, "num_splits": splits,
+            "ms_per_step": ms, "steps": steps, "tflops": tf, "bound": "tensor",
+            "peak_tflops": float(peaks["bf16_tflops"]), "frac": tf / float(peaks["bf16_tflops"]),
+            "kernel": "fused_attn_fwd_kernel<128, true>"}
 
 
 def main(argv=None):

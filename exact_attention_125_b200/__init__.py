@@ -17,6 +17,7 @@ import threading
 
 __all__ = [
     "AttnError", "lib", "attn_fwd", "attn_fwd_kv", "kv_num_splits", "kv_workspace_bytes",
+    "attn_fwd_ext", "ext_num_splits", "ext_workspace_bytes",
     "attn_fwd_naive", "naive_workspace_bytes",
     "last_device_error", "status_string", "selftest_wait_timeout", "abi",
     "NOALLOC_SCRATCH_BYTES",
@@ -35,7 +36,7 @@ STATUS = {
     0: "ATTN_OK", -1: "ATTN_ERR_NULL", -2: "ATTN_ERR_SHAPE", -3: "ATTN_ERR_HEADDIM",
     -4: "ATTN_ERR_ALIGN", -5: "ATTN_ERR_SCALE", -6: "ATTN_ERR_CAUSAL",
     -7: "ATTN_ERR_WORKSPACE", -8: "ATTN_ERR_LAUNCH", -9: "ATTN_ERR_UNSUPPORTED_DEVICE",
-    -10: "ATTN_ERR_TIMEOUT", -11: "ATTN_ERR_CUDA",
+    -10: "ATTN_ERR_TIMEOUT", -11: "ATTN_ERR_CUDA", -12: "ATTN_ERR_WINDOW",
 }
 
 
@@ -65,6 +66,13 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_kv_num_splits.restype = i
         L.attn_fwd_kv_workspace_bytes.argtypes = [i, i, i, i, i, i]
         L.attn_fwd_kv_workspace_bytes.restype = sz
+        L.attn_fwd_ext.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, i, vp, sz,
+                                   vp]
+        L.attn_fwd_ext.restype = i
+        L.attn_fwd_ext_num_splits.argtypes = [i, i, i, i, i, i]
+        L.attn_fwd_ext_num_splits.restype = i
+        L.attn_fwd_ext_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.attn_fwd_ext_workspace_bytes.restype = sz
         L.attn_fwd_naive_workspace_bytes.argtypes = [i, i, i]
         L.attn_fwd_naive_workspace_bytes.restype = sz
         L.attn_fwd_naive.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
@@ -103,6 +111,20 @@ class abi:
     @staticmethod
     def attn_fwd_kv_workspace_bytes(B, H, Nq, Nk, d, num_splits) -> int:
         return int(lib().attn_fwd_kv_workspace_bytes(B, H, Nq, Nk, d, num_splits))
+
+    @staticmethod
+    def attn_fwd_ext(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, window_left, window_right,
+                     alibi_slopes, num_splits, ws, ws_bytes, stream) -> int:
+        return lib().attn_fwd_ext(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, window_left,
+                                  window_right, alibi_slopes, num_splits, ws, ws_bytes, stream)
+
+    @staticmethod
+    def attn_fwd_ext_num_splits(B, H, Nq, Nk, d, window_left) -> int:
+        return lib().attn_fwd_ext_num_splits(B, H, Nq, Nk, d, window_left)
+
+    @staticmethod
+    def attn_fwd_ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits) -> int:
+        return int(lib().attn_fwd_ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits))
 
     @staticmethod
     def attn_fwd_naive(q, k, v, o, lse, B, H, N, d, scale, causal, ws, ws_bytes, stream) -> int:
@@ -218,6 +240,57 @@ def attn_fwd_kv(q, k, v, o=None, lse=None, scale=None, causal=False, num_splits=
                          ws_bytes, _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_kv")
+    return o, lse
+
+
+def ext_num_splits(B: int, H: int, Nq: int, Nk: int, d: int, window_left: int = -1) -> int:
+    st = abi.attn_fwd_ext_num_splits(B, H, Nq, Nk, d, window_left)
+    if st < 1:
+        raise AttnError(st, "attn_fwd_ext_num_splits")
+    return st
+
+
+def ext_workspace_bytes(B: int, H: int, Nq: int, Nk: int, d: int, window_left: int = -1,
+                        num_splits: int = 0) -> int:
+    return abi.attn_fwd_ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits)
+
+
+def attn_fwd_ext(q, k, v, o=None, lse=None, scale=None, causal=False, window_left=-1,
+                 window_right=-1, alibi_slopes=None, num_splits=0, workspace=None, stream=None):
+    """attn_fwd_kv with a key window [pos - window_left, pos + window_right]
+    around each query's position (-1 = unbounded) and an optional per-head
+    linear distance bias (alibi_slopes: CUDA fp32 tensor of H slopes; the
+    logit of key j drops by slope * |pos - j|). Returns (o, lse)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous bf16 [B, H, N, d] tensor")
+    if k.shape != v.shape or k.shape[:2] != q.shape[:2] or k.shape[3] != q.shape[3]:
+        raise ValueError("q [B, H, Nq, d] and k, v [B, H, Nk, d] expected")
+    B, H, Nq, d = (int(x) for x in q.shape)
+    Nk = int(k.shape[2])
+    sl_ptr = None
+    if alibi_slopes is not None:
+        if (not isinstance(alibi_slopes, torch.Tensor) or not alibi_slopes.is_cuda or
+                alibi_slopes.dtype != torch.float32 or alibi_slopes.numel() != H or
+                not alibi_slopes.is_contiguous()):
+            raise TypeError("alibi_slopes must be a contiguous CUDA float32 tensor of H values")
+        sl_ptr = alibi_slopes.data_ptr()
+    o, lse = _outputs(q, o, lse)
+    need = ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = abi.attn_fwd_ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, H, Nq, Nk, d, scale, int(bool(causal)), int(window_left),
+                          int(window_right), sl_ptr, int(num_splits), ws_ptr, ws_bytes,
+                          _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_ext")
     return o, lse
 
 

@@ -80,3 +80,21 @@ def kv_flops(B: int, H: int, Nq: int, Nk: int, d: int, causal: bool) -> float:
 
 def kv_bytes(B: int, H: int, Nq: int, Nk: int, d: int) -> int:
     return 2 * B * H * (2 * Nq + 2 * Nk) * d + 4 * B * H * Nq
+
+
+def ext_visible_pairs(Nq: int, Nk: int, causal: bool, window_left: int = -1,
+                      window_right: int = -1) -> int:
+    """(query, key) pairs allowed by the causal rule and a key window
+    [pos - window_left, pos + window_right] around pos = i + Nk - Nq, per head."""
+    total = 0
+    off = Nk - Nq
+    for i in range(Nq):
+        pos = i + off
+        hi = Nk - 1
+        if causal:
+            hi = min(hi, pos)
+        if window_right >= 0:
+            hi = min(hi, pos + window_right)
+        lo = max(0, pos - window_left) if window_left >= 0 else 0
+        total += max(0, hi - lo + 1)
+    return total

@@ -109,7 +109,8 @@ int sm_count(int* sms) {
 
 // Requested split count -> effective plan; num_splits = 0 asks for the
 // automatic choice on the current device.
-int resolve_kv_plan(int B, int H, int Nq, int Nk, int num_splits, attn::KvPlan* plan) {
+int resolve_kv_plan(int B, int H, int Nq, int Nk, int num_splits, int window_left,
+                    attn::KvPlan* plan) {
   if (num_splits < 0 || num_splits > attn::kMaxKvSplits) return ATTN_ERR_SHAPE;
   const int BH = B * H;
   if (num_splits == 0) {
@@ -117,25 +118,26 @@ int resolve_kv_plan(int B, int H, int Nq, int Nk, int num_splits, attn::KvPlan* 
     if (st != ATTN_OK) return st;
     int sms = 0;
     if ((st = sm_count(&sms)) != ATTN_OK) return st;
-    num_splits = attn::default_kv_splits(BH, Nq, Nk, sms);
+    num_splits = attn::default_kv_splits(BH, Nq, Nk, sms, window_left);
   }
-  *plan = attn::plan_kv(BH, Nq, Nk, num_splits);
+  *plan = attn::plan_kv(BH, Nq, Nk, num_splits, window_left);
   return ATTN_OK;
 }
 
-}  // namespace
-
-int attn_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                int Nq, int Nk, int d, float scale, int causal, int num_splits, void* workspace,
-                size_t workspace_bytes, attn_stream_t stream) {
+int fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+            int Nq, int Nk, int d, float scale, int causal, int window_left, int window_right,
+            const float* slopes, int num_splits, void* workspace, size_t workspace_bytes,
+            attn_stream_t stream) {
   int st = validate_kv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal);
   if (st != ATTN_OK) return st;
+  if (window_left < -1 || window_right < -1) return ATTN_ERR_WINDOW;
+  if (slopes && !aligned(slopes, 4)) return ATTN_ERR_ALIGN;
   if (num_splits < 0 || num_splits > attn::kMaxKvSplits) return ATTN_ERR_SHAPE;
   // An explicit split count is checked against the workspace before the
   // device is touched; the automatic one needs the device's SM count.
   if (num_splits == 0 && (st = check_device()) != ATTN_OK) return st;
   attn::KvPlan plan{};
-  if ((st = resolve_kv_plan(B, H, Nq, Nk, num_splits, &plan)) != ATTN_OK) return st;
+  if ((st = resolve_kv_plan(B, H, Nq, Nk, num_splits, window_left, &plan)) != ATTN_OK) return st;
   const size_t need = attn::kv_workspace_bytes(B * H, Nq, d, plan.nsplit);
   if (need > 0) {
     if (!workspace) return ATTN_ERR_NULL;
@@ -156,21 +158,59 @@ int attn_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse
   a.d = d;
   a.scale = scale;
   a.causal = causal;
+  a.window_left = window_left;
+  a.window_right = window_right;
+  a.slopes = slopes;
   return attn::launch_fused_kv(a, plan, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int attn_fwd_kv_num_splits(int B, int H, int Nq, int Nk, int d) {
-  if (!kv_shape_ok(B, H, Nq, Nk, d)) return ATTN_ERR_SHAPE;
+int ext_num_splits(int B, int H, int Nq, int Nk, int d, int window_left) {
+  if (!kv_shape_ok(B, H, Nq, Nk, d) || window_left < -1) return ATTN_ERR_SHAPE;
   attn::KvPlan plan{};
-  const int st = resolve_kv_plan(B, H, Nq, Nk, 0, &plan);
+  const int st = resolve_kv_plan(B, H, Nq, Nk, 0, window_left, &plan);
   return st != ATTN_OK ? st : plan.nsplit;
 }
 
-size_t attn_fwd_kv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits) {
-  if (!kv_shape_ok(B, H, Nq, Nk, d)) return 0;
+size_t ext_workspace_bytes(int B, int H, int Nq, int Nk, int d, int window_left,
+                           int num_splits) {
+  if (!kv_shape_ok(B, H, Nq, Nk, d) || window_left < -1) return 0;
   attn::KvPlan plan{};
-  if (resolve_kv_plan(B, H, Nq, Nk, num_splits, &plan) != ATTN_OK) return 0;
+  if (resolve_kv_plan(B, H, Nq, Nk, num_splits, window_left, &plan) != ATTN_OK) return 0;
   return attn::kv_workspace_bytes(B * H, Nq, d, plan.nsplit);
+}
+
+}  // namespace
+
+int attn_fwd_kv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int Nq, int Nk, int d, float scale, int causal, int num_splits, void* workspace,
+                size_t workspace_bytes, attn_stream_t stream) {
+  return fwd_ext(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, -1, -1, nullptr, num_splits,
+                 workspace, workspace_bytes, stream);
+}
+
+int attn_fwd_kv_num_splits(int B, int H, int Nq, int Nk, int d) {
+  return ext_num_splits(B, H, Nq, Nk, d, -1);
+}
+
+size_t attn_fwd_kv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits) {
+  return ext_workspace_bytes(B, H, Nq, Nk, d, -1, num_splits);
+}
+
+int attn_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int Nq, int Nk, int d, float scale, int causal, int window_left,
+                 int window_right, const float* alibi_slopes, int num_splits, void* workspace,
+                 size_t workspace_bytes, attn_stream_t stream) {
+  return fwd_ext(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, window_left, window_right,
+                 alibi_slopes, num_splits, workspace, workspace_bytes, stream);
+}
+
+int attn_fwd_ext_num_splits(int B, int H, int Nq, int Nk, int d, int window_left) {
+  return ext_num_splits(B, H, Nq, Nk, d, window_left);
+}
+
+size_t attn_fwd_ext_workspace_bytes(int B, int H, int Nq, int Nk, int d, int window_left,
+                                    int num_splits) {
+  return ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits);
 }
 
 size_t attn_fwd_naive_workspace_bytes(int B, int H, int N) {
@@ -248,6 +288,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_UNSUPPORTED_DEVICE: return "ATTN_ERR_UNSUPPORTED_DEVICE: needs an sm_100 GPU";
     case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT: a device-side bounded wait ran out";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA runtime call failed";
+    case ATTN_ERR_WINDOW: return "ATTN_ERR_WINDOW: a window bound is below -1";
     default: return "unknown attn status";
   }
 }

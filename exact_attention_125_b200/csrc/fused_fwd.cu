@@ -124,6 +124,10 @@ struct FwdParams {
   int alt;       // 1: one query tile per CTA, the two softmax warpgroups take alternate KV tiles
   float* part_o;    // [nsplit][BH][Nq][D] fp32, normalised per split (nsplit > 1)
   float* part_lse;  // [nsplit][BH][Nq] fp32 natural-log lse per split (nsplit > 1)
+  int t_begin;      // first KV tile any query row needs (the splits cut [t_begin, T))
+  int wl, wr;       // key window [pos - wl, pos + wr] around query position pos; < 0: unbounded
+  int H;
+  const float* slopes;  // per-head linear distance bias slopes (natural log units), or null
 };
 
 // What one CTA of the kv path works on.
@@ -148,22 +152,28 @@ __device__ __forceinline__ KvWork kv_work_of(const FwdParams& p, int& bh, int& q
   const int r = rem % p.nqb;
   const int qblk = p.causal ? (p.nqb - 1 - r) : r;
   q0 = qblk * (p.alt ? kTileRows : kBlockRows);
-  kw.kv_lo = kw.split * p.tps;
-  const int kv_hi = min(p.T, kw.kv_lo + p.tps);
-  // KV tiles up to the last one that some row of the tile starting at r0 sees
+  const int s_lo = p.t_begin + kw.split * p.tps;  // this split's KV tiles [s_lo, s_hi)
+  const int s_hi = min(p.T, s_lo + p.tps);
+  // one past the last KV tile that some row of the tile starting at r0 sees
   auto need = [&](int r0) -> int {
     if (r0 >= p.Nq) return 0;
-    if (!p.causal) return p.T;
     const int r1 = min(r0 + kTileRows - 1, p.Nq - 1);
-    return min(p.T, (r1 + p.offset) / kTileRows + 1);
+    long long hi = p.N - 1;
+    if (p.causal) hi = min(hi, static_cast<long long>(r1) + p.offset);
+    if (p.wr >= 0) hi = min(hi, static_cast<long long>(r1) + p.offset + p.wr);
+    return hi < 0 ? 0 : static_cast<int>(hi / kTileRows) + 1;
   };
+  // first KV tile the first row of the CTA sees (a left window bound)
+  const long long first_key =
+      p.wl >= 0 ? max(0ll, static_cast<long long>(q0) + p.offset - p.wl) : 0ll;
+  kw.kv_lo = max(s_lo, static_cast<int>(first_key / kTileRows));
   if (p.alt) {
-    const int n = max(0, min(kv_hi, need(q0)) - kw.kv_lo);
+    const int n = max(0, min(s_hi, need(q0)) - kw.kv_lo);
     kw.na = (n + 1) / 2;
     kw.nb = n / 2;
   } else {
-    kw.na = max(0, min(kv_hi, need(q0)) - kw.kv_lo);
-    kw.nb = max(0, min(kv_hi, need(q0 + kTileRows)) - kw.kv_lo);
+    kw.na = max(0, min(s_hi, need(q0)) - kw.kv_lo);
+    kw.nb = max(0, min(s_hi, need(q0 + kTileRows)) - kw.kv_lo);
   }
   return kw;
 }
@@ -204,6 +214,29 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
   const int row_start = alt ? q0 : q0 + kTileRows * g;
   const int row = row_start + tid;
   const float c = p.scale_log2;
+  // kv path: this row's allowed keys [key_lo, key_hi] (causal limit, window,
+  // key count); the tile's first row has the lowest key_hi and its last row
+  // the highest key_lo, which decide whether a KV tile needs masking at all.
+  int key_lo = 0, key_hi = p.N - 1, tile_hi = p.N - 1, tile_lo = 0;
+  float slope_l2 = 0.0f;
+  if constexpr (kKV) {
+    auto hi_of = [&](int r) {
+      long long h = p.N - 1;
+      if (p.causal) h = min(h, static_cast<long long>(r) + p.offset);
+      if (p.wr >= 0) h = min(h, static_cast<long long>(r) + p.offset + p.wr);
+      return static_cast<int>(max(h, -1ll));
+    };
+    auto lo_of = [&](int r) {
+      return p.wl >= 0 ? static_cast<int>(min(max(0ll, static_cast<long long>(r) + p.offset - p.wl),
+                                              static_cast<long long>(p.N)))
+                       : 0;
+    };
+    key_hi = hi_of(row);
+    key_lo = lo_of(row);
+    tile_hi = hi_of(row_start);
+    tile_lo = lo_of(row_start + kTileRows - 1);
+    if (p.slopes) slope_l2 = p.slopes[bh % p.H] * 1.4426950408889634f;
+  }
 
   float m_run = -INFINITY;
   float l_run = 0.0f;
@@ -216,19 +249,36 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
 
     bool need_mask;
     int col0;
+    float cs = c;  // multiplier from the values in sr to log2-domain logits
     if constexpr (kKV) {
       col0 = (kv_lo + (alt ? 2 * j + g : j)) * kTileRows;
-      need_mask = (p.causal && col0 + kTileRows - 1 > row_start + p.offset) || (col0 + kTileRows > p.N);
+      need_mask = (col0 + kTileRows - 1 > tile_hi) || (col0 < tile_lo);
+      if (need_mask) {
+        const int lim_hi = key_hi - col0;
+        const int lim_lo = key_lo - col0;
+#pragma unroll
+        for (int cc = 0; cc < 128; ++cc)
+          if (cc > lim_hi || cc < lim_lo) sr[cc] = 0xff800000u;  // -inf
+      }
+      if (p.slopes) {
+        // linear distance bias: x = s * c - slope * log2(e) * |pos - key|
+        const float rel = static_cast<float>(row + p.offset - col0);
+#pragma unroll
+        for (int cc = 0; cc < 128; ++cc)
+          sr[cc] = __float_as_uint(
+              fmaf(__uint_as_float(sr[cc]), c, -slope_l2 * fabsf(rel - static_cast<float>(cc))));
+        cs = 1.0f;
+      }
     } else {
       col0 = j * kTileRows;
       need_mask = (p.causal && col0 + kTileRows - 1 > row_start) || (col0 + kTileRows > p.N);
-    }
-    if (need_mask) {
-      int lim = p.N - 1 - col0;
-      if (p.causal) lim = min(lim, row + (kKV ? p.offset : 0) - col0);
+      if (need_mask) {
+        int lim = p.N - 1 - col0;
+        if (p.causal) lim = min(lim, row - col0);
 #pragma unroll
-      for (int cc = 0; cc < 128; ++cc)
-        if (cc > lim) sr[cc] = 0xff800000u;  // -inf
+        for (int cc = 0; cc < 128; ++cc)
+          if (cc > lim) sr[cc] = 0xff800000u;  // -inf
+      }
     }
 
     float mx[8];
@@ -239,7 +289,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
       mx[(cc / 2) % 8] = fmax3(mx[(cc / 2) % 8], __uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1]));
     const float rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
                              fmaxf(mx[6], mx[7]));
-    const float m_tile = rmax * c;
+    const float m_tile = rmax * cs;
     const bool raise = m_tile > m_run + kRescaleThreshold;
     const float m_new = raise ? m_tile : m_run;
     const float alpha = raise ? ex2_approx(m_run - m_new) : 1.0f;
@@ -261,7 +311,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     // p = 2^(s * c - m) for the 64 (even, odd) column pairs: scaling and
     // summing in packed f32x2 form; most exponentials on the MUFU (ex2), the
     // pairs poly_pair picks on the FMA pipe (exp2_poly_pair).
-    const uint64_t c2 = f2_pack(c, c);
+    const uint64_t c2 = f2_pack(cs, cs);
     const uint64_t nm2 = f2_pack(neg_m, neg_m);
     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
     uint32_t pk[64];
@@ -950,6 +1000,11 @@ int launch_fused_kv_d(const AttnKvArgs& a, const KvPlan& plan, void* workspace,
   p.nsplit = plan.nsplit;
   p.tps = plan.tps;
   p.alt = plan.alt;
+  p.t_begin = plan.t_begin;
+  p.wl = a.window_left;
+  p.wr = a.window_right;
+  p.H = a.H;
+  p.slopes = a.slopes;
   if (plan.nsplit > 1) {
     p.part_o = static_cast<float*>(workspace);
     p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -973,28 +1028,34 @@ int launch_fused_kv_d(const AttnKvArgs& a, const KvPlan& plan, void* workspace,
 
 }  // namespace
 
-KvPlan plan_kv(int BH, int Nq, int Nk, int num_splits) {
+KvPlan plan_kv(int BH, int Nq, int Nk, int num_splits, int window_left) {
   KvPlan pl{};
   pl.T = (Nk + kTileRows - 1) / kTileRows;
   pl.alt = Nq <= kTileRows ? 1 : 0;
   pl.nqb = (Nq + (pl.alt ? kTileRows : kBlockRows) - 1) / (pl.alt ? kTileRows : kBlockRows);
-  const int s = std::max(1, std::min(num_splits, pl.T));
-  pl.tps = (pl.T + s - 1) / s;
-  pl.nsplit = (pl.T + pl.tps - 1) / pl.tps;  // no empty split
+  // keys before the first query row's window are never read: the splits cut
+  // [t_begin, T) (query row 0 is sequence position Nk - Nq)
+  const long long first_key =
+      window_left >= 0 ? std::max(0ll, static_cast<long long>(Nk) - Nq - window_left) : 0ll;
+  pl.t_begin = static_cast<int>(std::min<long long>(first_key / kTileRows, pl.T - 1));
+  const int len = pl.T - pl.t_begin;
+  const int s = std::max(1, std::min(num_splits, len));
+  pl.tps = (len + s - 1) / s;
+  pl.nsplit = (len + pl.tps - 1) / pl.tps;  // no empty split
   (void)BH;
   return pl;
 }
 
-int default_kv_splits(int BH, int Nq, int Nk, int sms) {
-  const KvPlan one = plan_kv(BH, Nq, Nk, 1);
+int default_kv_splits(int BH, int Nq, int Nk, int sms, int window_left) {
+  const KvPlan one = plan_kv(BH, Nq, Nk, 1, window_left);
   const long long base = static_cast<long long>(BH) * one.nqb;
   if (sms < 1 || base >= sms) return 1;
   // At least kMinTilesPerSplit KV tiles per CTA keeps the per-CTA start-up
   // (Q load, pipeline fill, epilogue) small against its streaming time.
   constexpr int kMinTilesPerSplit = 8;
-  const int max_s = std::max(1, std::min(kMaxKvSplits, one.T / kMinTilesPerSplit));
+  const int max_s = std::max(1, std::min(kMaxKvSplits, (one.T - one.t_begin) / kMinTilesPerSplit));
   auto eff = [&](int s) {
-    const long long n = base * plan_kv(BH, Nq, Nk, s).nsplit;
+    const long long n = base * plan_kv(BH, Nq, Nk, s, window_left).nsplit;
     const long long waves = (n + sms - 1) / sms;
     return static_cast<double>(n) / static_cast<double>(waves * sms);
   };
@@ -1002,7 +1063,7 @@ int default_kv_splits(int BH, int Nq, int Nk, int sms) {
   for (int s = 1; s <= max_s; ++s) best = std::max(best, eff(s));
   // the fewest splits within 15% of the best wave efficiency
   for (int s = 1; s <= max_s; ++s)
-    if (eff(s) >= 0.85 * best) return plan_kv(BH, Nq, Nk, s).nsplit;
+    if (eff(s) >= 0.85 * best) return plan_kv(BH, Nq, Nk, s, window_left).nsplit;
   return 1;
 }
 

@@ -32,6 +32,8 @@ struct AttnKvArgs {
   int B, H, Nq, Nk, d;
   float scale;
   int causal;
+  int window_left, window_right;  // key window around the query position; < 0: unbounded
+  const float* slopes;            // per-head linear distance bias slopes (device), or null
 };
 
 // How the kv path cuts the work: T KV tiles of 128 keys, tps tiles per split,
@@ -39,14 +41,16 @@ struct AttnKvArgs {
 // (one query tile per CTA, its two softmax warpgroups on alternate KV tiles).
 struct KvPlan {
   int T, tps, nsplit, alt, nqb;
+  int t_begin;  // first KV tile any query row needs; the splits cut [t_begin, T)
 };
 
 constexpr int kMaxKvSplits = 256;
 
-// Plan for a requested split count (clamped to [1, T]).
-KvPlan plan_kv(int BH, int Nq, int Nk, int num_splits);
+// Plan for a requested split count (clamped to [1, T - t_begin]); window_left
+// < 0 means no left window bound.
+KvPlan plan_kv(int BH, int Nq, int Nk, int num_splits, int window_left);
 // Split count the library picks for a GPU with `sms` multiprocessors.
-int default_kv_splits(int BH, int Nq, int Nk, int sms);
+int default_kv_splits(int BH, int Nq, int Nk, int sms, int window_left);
 // Bytes of the fp32 partial-O block (rounded up to 256) and of the whole
 // workspace (partial O, then partial lse) for nsplit splits; 0 when nsplit <= 1.
 size_t kv_partial_o_bytes(int BH, int Nq, int d, int nsplit);

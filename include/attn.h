@@ -67,7 +67,8 @@ enum {
     ATTN_ERR_LAUNCH = -8,             /* the CUDA launch failed */
     ATTN_ERR_UNSUPPORTED_DEVICE = -9, /* current device is not sm_100 */
     ATTN_ERR_TIMEOUT = -10,           /* a kernel gave up on a bounded wait */
-    ATTN_ERR_CUDA = -11               /* another CUDA runtime/driver call failed */
+    ATTN_ERR_CUDA = -11,              /* another CUDA runtime/driver call failed */
+    ATTN_ERR_WINDOW = -12             /* attn_fwd_ext: a window bound below -1 */
 };
 
 /*
@@ -139,6 +140,45 @@ int attn_fwd_kv_num_splits(int B, int H, int Nq, int Nk, int d);
  */
 size_t attn_fwd_kv_workspace_bytes(int B, int H, int Nq, int Nk, int d,
                                    int num_splits);
+
+/*
+ * attn_fwd_ext - attn_fwd_kv with the variants a fused library usually does
+ * not cover (anylearn.cc, "Attention Is Memory-Bound, and Nobody Noticed for
+ * Five Years": "a custom attention bias, an unusual masking pattern, a novel
+ * position encoding" fall off the fast path), computed inside the same fused
+ * kernel:
+ *
+ * - a key window around the query's sequence position pos = i + (Nk - Nq):
+ *   key j is allowed iff pos - window_left <= j (when window_left >= 0) and
+ *   j <= pos + window_right (when window_right >= 0), on top of the causal
+ *   rule; -1 leaves that side unbounded. causal = 1 with window_left = W - 1
+ *   is a sliding window of the W most recent keys. KV tiles wholly outside
+ *   every row's window are never loaded.
+ * - alibi_slopes: NULL, or H device floats (4-byte aligned, finite); the
+ *   logit of key j for a query at position pos becomes
+ *   scale * q.k_j - alibi_slopes[h] * |pos - j| (a per-head linear distance
+ *   bias; natural-log units, added after the scale).
+ *
+ * A row with no allowed key gets O = 0 and lse = -inf. Other arguments,
+ * layouts and the split / workspace rules as for attn_fwd_kv, except that the
+ * splits cut only the key tiles from the first row's window start on; size
+ * the workspace with attn_fwd_ext_workspace_bytes. ATTN_ERR_WINDOW if a
+ * window bound is below -1.
+ */
+int attn_fwd_ext(const void *q, const void *k, const void *v, void *o,
+                 float *lse, int B, int H, int Nq, int Nk, int d, float scale,
+                 int causal, int window_left, int window_right,
+                 const float *alibi_slopes, int num_splits, void *workspace,
+                 size_t workspace_bytes, attn_stream_t stream);
+
+/* attn_fwd_ext_num_splits - the automatic split count of attn_fwd_ext on the
+ * current device (>= 1), or a negative ATTN_ERR_* code. */
+int attn_fwd_ext_num_splits(int B, int H, int Nq, int Nk, int d, int window_left);
+
+/* attn_fwd_ext_workspace_bytes - workspace attn_fwd_ext needs for num_splits
+ * (0 = automatic on the current device); 0 when one split or invalid. */
+size_t attn_fwd_ext_workspace_bytes(int B, int H, int Nq, int Nk, int d,
+                                    int window_left, int num_splits);
 
 /*
  * attn_fwd_naive_workspace_bytes - bytes of workspace attn_fwd_naive needs:

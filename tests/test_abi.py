@@ -125,3 +125,30 @@ def test_kv_workspace_bytes(L):
     assert f(1, 1, 3, 1000, 64, 7) == f(1, 1, 3, 1000, 64, 4)
     assert f(1, 1, 3, 1000, 64, 3) == 3 * 3 * 64 * 4 + 3 * 3 * 4 + (256 - (3 * 3 * 64 * 4) % 256) % 256
     assert f(0, 1, 3, 1000, 64, 3) == 0 and f(1, 1, 3, 1000, 96, 3) == 0
+
+
+def _ext(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=2, Nq=4, Nk=1000, d=64, scale=0.125,
+                causal=1, wl=127, wr=-1, slopes=None, splits=1, ws=None, ws_bytes=0, stream=None)
+    args.update(kw)
+    return ea.abi.attn_fwd_ext(*(args[n] for n in (
+        "q", "k", "v", "o", "lse", "B", "H", "Nq", "Nk", "d", "scale", "causal", "wl", "wr",
+        "slopes", "splits", "ws", "ws_bytes", "stream")))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(wl=-2), -12), (dict(wr=-5), -12), (dict(slopes=A + 2), -4), (dict(Nq=0), -2),
+    (dict(splits=3), -1), (dict(splits=3, ws=A, ws_bytes=10), -7),
+])
+def test_ext_argument_errors(L, kw, code):
+    assert _ext(**kw) == code
+
+
+def test_ext_workspace_counts_only_the_window():
+    f = ea.abi.attn_fwd_ext_workspace_bytes
+    # 1 query row at position 999 with a 127-key left window reads keys 872..999:
+    # tiles 6 and 7 only, so at most 2 splits
+    assert f(1, 2, 1, 1000, 64, 127, 8) == f(1, 2, 1, 1000, 64, 127, 2)
+    assert f(1, 2, 1, 1000, 64, 127, 2) == 2 * 2 * 64 * 4 + 2 * 2 * 4 + (256 - (2 * 2 * 64 * 4) % 256) % 256
+    assert f(1, 2, 1, 1000, 64, -1, 8) == ea.abi.attn_fwd_kv_workspace_bytes(1, 2, 1, 1000, 64, 8)
+    assert f(1, 2, 1, 1000, 64, -2, 8) == 0

@@ -144,3 +144,20 @@ def test_kv_inputs_shapes_and_determinism():
     assert q.shape == (1, 2, 3, 8) and k.shape == v.shape == (1, 2, 7, 8)
     q2, k2, v2 = make_q_kv(1, 2, 3, 7, 8, seed=5)
     assert torch.equal(q, q2) and torch.equal(k, k2) and torch.equal(v, v2)
+
+
+@pytest.mark.parametrize("Nq,Nk,causal,wl,wr", [(5, 9, True, 2, -1), (7, 7, False, 1, 3),
+                                                (3, 12, False, -1, 0), (6, 6, True, -1, -1)])
+def test_ext_visible_pairs_count_the_mask(Nq, Nk, causal, wl, wr):
+    pos = np.arange(Nq)[:, None] + (Nk - Nq)
+    j = np.arange(Nk)[None, :]
+    ok = np.ones((Nq, Nk), dtype=bool)
+    if causal:
+        ok &= j <= pos
+    if wl >= 0:
+        ok &= j >= pos - wl
+    if wr >= 0:
+        ok &= j <= pos + wr
+    assert costs.ext_visible_pairs(Nq, Nk, causal, wl, wr) == int(ok.sum())
+    if wl < 0 and wr < 0:
+        assert costs.ext_visible_pairs(Nq, Nk, causal) == costs.kv_visible_pairs(Nq, Nk, causal)

@@ -1,0 +1,79 @@
+"""attn_fwd_ext (key windows around the query position and a per-head linear
+distance bias, inside the fused kernel) against the fp64 oracle, element by
+element on every row. Covers sliding windows (causal with a left bound),
+two-sided windows without the causal rule, a window of one key, the distance
+bias alone and together with a window, decode and prefill shapes, both CTA
+layouts, explicit and automatic split counts, and rows with no allowed key
+(O = 0, lse = -inf on both sides).
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_125_b200 as ea
+import oracle
+from exact_attention_125_b200.inputs import gather_rows, make_q_kv
+from parity_util import assert_within, compare, scale_of
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # B, H, Nq, Nk, d, causal, window_left, window_right, slopes, num_splits
+    (1, 2, 300, 300, 128, True, 63, -1, None, 1),
+    (1, 2, 300, 300, 64, True, 200, -1, "alibi", 1),
+    (2, 2, 1, 5000, 128, True, 1000, -1, None, 0),
+    (1, 4, 1, 3000, 128, False, -1, -1, "alibi", 3),
+    (1, 2, 100, 1100, 128, True, 300, -1, "steep", 4),
+    (1, 2, 129, 700, 64, False, 100, 50, None, 2),
+    (1, 1, 600, 600, 128, False, 0, 0, None, 1),
+    (1, 2, 256, 256, 128, True, -1, -1, "alibi", 1),
+    (1, 2, 500, 2000, 128, True, 127, -1, None, 5),
+    (1, 2, 700, 700, 128, True, 255, -1, "steep", 0),
+    (1, 1, 300, 200, 64, False, 10, 10, None, 1),   # early rows: no key in their window
+    (1, 3, 17, 4096, 64, True, 511, -1, "alibi", 0),
+]
+
+
+def _slopes(kind, H):
+    if kind is None:
+        return None
+    if kind == "alibi":  # the geometric slopes 2^(-8 (h + 1) / H)
+        return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
+    return [0.5 / (h + 1) for h in range(H)]  # steep: a few keys dominate
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d,causal,wl,wr,kind,splits", CASES)
+def test_ext_all_rows(B, H, Nq, Nk, d, causal, wl, wr, kind, splits):
+    q, k, v = make_q_kv(B, H, Nq, Nk, d, seed=Nq * 13 + Nk + wl + 7 * wr + d)
+    slopes = _slopes(kind, H)
+    qg, kg, vg = (t.to("cuda") for t in (q, k, v))
+    sl = torch.tensor(slopes, dtype=torch.float32, device="cuda") if slopes else None
+    o = torch.full((B, H, Nq, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, H, Nq), float("nan"), dtype=torch.float32, device="cuda")
+    ea.attn_fwd_ext(qg, kg, vg, o, lse, scale=scale_of(d), causal=causal, window_left=wl,
+                    window_right=wr, alibi_slopes=sl, num_splits=splits)
+    torch.cuda.synchronize()
+    assert ea.last_device_error() == 0
+    rows = oracle.all_rows(B * H, Nq)
+    # the oracle gets the fp32 slopes the kernel uses, widened exactly
+    sl64 = [float(np.float32(x)) for x in slopes] if slopes else None
+    o_ref, lse_ref = oracle.attention_ext(q, k, v, scale_of(d), causal, wl, wr, sl64, rows=rows)
+    o_rows = gather_rows(o.cpu(), rows)
+    lse_rows = gather_rows(lse.cpu().unsqueeze(-1), rows).squeeze(-1)
+    empty = np.isneginf(lse_ref)
+    if empty.any():
+        assert np.isneginf(lse_rows.numpy()[empty]).all()
+        assert (o_rows.float().numpy()[empty] == 0).all()
+    keep = ~empty
+    e = compare(o_rows[torch.as_tensor(keep)], lse_rows[torch.as_tensor(keep)], o_ref[keep],
+                lse_ref[keep])
+    assert_within(e, f"{(B, H, Nq, Nk, d, causal, wl, wr, kind, splits)}")
+
+
+def test_ext_without_options_matches_attn_fwd_kv_bit_for_bit():
+    q, k, v = make_q_kv(1, 2, 40, 3000, 128, seed=9)
+    qg, kg, vg = (t.to("cuda") for t in (q, k, v))
+    o1, l1 = ea.attn_fwd_kv(qg, kg, vg, causal=True, num_splits=3)
+    o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=True, num_splits=3)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
