@@ -55,6 +55,7 @@ def parse_args(argv=None):
     p.add_argument("--no-naive", action="store_true", help="skip the unfused traffic line")
     p.add_argument("--no-kv", action="store_true", help="skip the split-KV inference lines")
     p.add_argument("--no-ext", action="store_true", help="skip the window / distance-bias lines")
+    p.add_argument("--no-chain", action="store_true", help="skip the elementwise-chain line")
     p.add_argument("--kv-only", default=None, metavar="WORKLOAD",
                    help="run only the split-KV line of this inference workload (one GPU)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -365,6 +366,7 @@ def run_ours(args):
     split_kv = None if args.no_kv else [split_kv_line(name, device, peaks)
                                        for name in KV_BENCH_WORKLOADS]
     ext = None if args.no_ext else [ext_line(spec, device, peaks) for spec in EXT_BENCH]
+    chain = None if args.no_chain else chain_line(device, peaks)
 
     peak = float(peaks["bf16_tflops"])
     line = {
@@ -411,6 +413,8 @@ def run_ours(args):
         line["split_kv"] = split_kv
     if ext is not None:
         line["masks_and_bias"] = ext
+    if chain is not None:
+        line["elementwise_chain"] = chain
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, n, cores, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -629,6 +633,46 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
             "ms_per_step": ms, "steps": steps, "tflops": tf, "bound": "tensor",
             "peak_tflops": float(peaks["bf16_tflops"]), "frac": tf / float(peaks["bf16_tflops"]),
             "kernel": "fused_attn_fwd_kernel<128, true>"}
+
+
+def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
+    """y = gelu(0.5 x + b) over a [65536, 8192] bf16 tensor (1 GiB, above L2),
+    one fused kernel against three: achieved GB/s of each path's own traffic
+    (fused: x read, y written; unfused: three reads and three writes) and the
+    time ratio the page predicts to be about 3."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    g = torch.Generator(device=device).manual_seed(77)
+    x = torch.randn((rows, cols), device=device, generator=g).to(torch.bfloat16)
+    b = torch.randn((cols,), device=device, generator=g).to(torch.bfloat16)
+    y = torch.empty_like(x)
+    tmp = torch.empty_like(x)
+    stream = torch.cuda.current_stream(device)
+    out = {}
+    for name, fn in (("fused", lambda: ea.chain_fused(x, b, y, 0.5, "gelu", stream)),
+                     ("unfused", lambda: ea.chain_unfused(x, b, y, tmp, 0.5, "gelu", stream))):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(steps):
+            fn()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        ms = start.elapsed_time(end) / steps
+        nbytes = (2 if name == "fused" else 6) * rows * cols * 2 + cols * 2
+        out[name] = {"ms_per_step": ms, "algorithmic_bytes": nbytes,
+                     "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "frac": nbytes / (ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                     "launches_per_step": 1 if name == "fused" else 3}
+    del x, y, tmp
+    torch.cuda.empty_cache()
+    return {"workload": f"gelu(0.5 x + b), x [{rows}, {cols}] bf16", "bound": "hbm",
+            "hbm_peak_gbs": float(peaks["hbm_gbs"]), **out,
+            "speedup_fused_over_unfused": out["unfused"]["ms_per_step"] / out["fused"]["ms_per_step"],
+            "kernel": "chain_pass_kernel"}
 
 
 def main(argv=None):

@@ -17,7 +17,8 @@ import threading
 
 __all__ = [
     "AttnError", "lib", "attn_fwd", "attn_fwd_kv", "kv_num_splits", "kv_workspace_bytes",
-    "attn_fwd_ext", "ext_num_splits", "ext_workspace_bytes",
+    "attn_fwd_ext", "ext_num_splits", "ext_workspace_bytes", "chain_fused", "chain_unfused",
+    "CHAIN_ACTS",
     "attn_fwd_naive", "naive_workspace_bytes",
     "last_device_error", "status_string", "selftest_wait_timeout", "abi",
     "NOALLOC_SCRATCH_BYTES",
@@ -73,6 +74,11 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_ext_num_splits.restype = i
         L.attn_fwd_ext_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
         L.attn_fwd_ext_workspace_bytes.restype = sz
+        ll = ctypes.c_longlong
+        L.chain_fused.argtypes = [vp, vp, vp, ll, i, f, i, vp]
+        L.chain_fused.restype = i
+        L.chain_unfused.argtypes = [vp, vp, vp, vp, ll, i, f, i, vp]
+        L.chain_unfused.restype = i
         L.attn_fwd_naive_workspace_bytes.argtypes = [i, i, i]
         L.attn_fwd_naive_workspace_bytes.restype = sz
         L.attn_fwd_naive.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
@@ -125,6 +131,14 @@ class abi:
     @staticmethod
     def attn_fwd_ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits) -> int:
         return int(lib().attn_fwd_ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits))
+
+    @staticmethod
+    def chain_fused(x, b, y, rows, cols, alpha, act, stream) -> int:
+        return lib().chain_fused(x, b, y, rows, cols, alpha, act, stream)
+
+    @staticmethod
+    def chain_unfused(x, b, y, tmp, rows, cols, alpha, act, stream) -> int:
+        return lib().chain_unfused(x, b, y, tmp, rows, cols, alpha, act, stream)
 
     @staticmethod
     def attn_fwd_naive(q, k, v, o, lse, B, H, N, d, scale, causal, ws, ws_bytes, stream) -> int:
@@ -292,6 +306,46 @@ def attn_fwd_ext(q, k, v, o=None, lse=None, scale=None, causal=False, window_lef
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_ext")
     return o, lse
+
+
+# CHAIN_ACT_* of include/chain.h
+CHAIN_ACTS = {"relu": 0, "gelu": 1, "silu": 2}
+
+
+def _check_chain(x, b):
+    import torch
+    for name, t in (("x", x), ("b", b)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 or \
+                not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA bf16 tensor")
+    if x.dim() != 2 or b.dim() != 1 or b.shape[0] != x.shape[1]:
+        raise ValueError("x [rows, cols] and b [cols] expected")
+    return int(x.shape[0]), int(x.shape[1])
+
+
+def chain_fused(x, b, y=None, alpha=1.0, act="gelu", stream=None):
+    """y = act(alpha * x + b) in one kernel (bf16 in and out)."""
+    import torch
+    rows, cols = _check_chain(x, b)
+    y = torch.empty_like(x) if y is None else y
+    st = abi.chain_fused(x.data_ptr(), b.data_ptr(), y.data_ptr(), rows, cols, float(alpha),
+                         CHAIN_ACTS[act], _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "chain_fused")
+    return y
+
+
+def chain_unfused(x, b, y=None, tmp=None, alpha=1.0, act="gelu", stream=None):
+    """The same chain as three kernels through a bf16 scratch tensor."""
+    import torch
+    rows, cols = _check_chain(x, b)
+    y = torch.empty_like(x) if y is None else y
+    tmp = torch.empty_like(x) if tmp is None else tmp
+    st = abi.chain_unfused(x.data_ptr(), b.data_ptr(), y.data_ptr(), tmp.data_ptr(), rows, cols,
+                           float(alpha), CHAIN_ACTS[act], _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "chain_unfused")
+    return y
 
 
 def naive_workspace_bytes(B: int, H: int, N: int) -> int:

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "../../include/chain.h"
 #include "internal.h"
 
 namespace {
@@ -251,6 +252,41 @@ int attn_fwd_naive_noalloc(const void* q, const void* k, const void* v, void* o,
   void* scratch = attn::noalloc_scratch_ptr();
   if (!scratch) return ATTN_ERR_CUDA;
   return attn::launch_naive(pack(q, k, v, o, lse, B, H, N, d, scale, causal), scratch,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+int validate_chain(const void* x, const void* b, const void* y, long long rows, int cols,
+                   float alpha, int act) {
+  if (!x || !b || !y) return ATTN_ERR_NULL;
+  if (rows < 1 || cols < 1 || cols % 8 != 0) return ATTN_ERR_SHAPE;
+  if (rows > (1ll << 62) / cols) return ATTN_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(b, 16) || !aligned(y, 16)) return ATTN_ERR_ALIGN;
+  if (!std::isfinite(alpha)) return ATTN_ERR_SCALE;
+  if (act < CHAIN_ACT_RELU || act > CHAIN_ACT_SILU) return ATTN_ERR_CAUSAL;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+int chain_fused(const void* x, const void* b, void* y, long long rows, int cols, float alpha,
+                int act, attn_stream_t stream) {
+  int st = validate_chain(x, b, y, rows, cols, alpha, act);
+  if (st != ATTN_OK) return st;
+  if ((st = check_device()) != ATTN_OK) return st;
+  return attn::launch_chain(x, b, y, nullptr, rows, cols, alpha, act, true,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int chain_unfused(const void* x, const void* b, void* y, void* tmp, long long rows, int cols,
+                  float alpha, int act, attn_stream_t stream) {
+  int st = validate_chain(x, b, y, rows, cols, alpha, act);
+  if (st != ATTN_OK) return st;
+  if (!tmp) return ATTN_ERR_NULL;
+  if (!aligned(tmp, 16)) return ATTN_ERR_ALIGN;
+  if ((st = check_device()) != ATTN_OK) return st;
+  return attn::launch_chain(x, b, y, tmp, rows, cols, alpha, act, false,
                             reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -64,6 +64,11 @@ int launch_fused_kv(const AttnKvArgs& a, const KvPlan& plan, void* workspace, cu
 int launch_lse_combine(const float* part_o, const float* part_lse, void* o, float* lse, int rows,
                        int d, int nsplit, cudaStream_t stream);
 
+// Elementwise chain y = act(alpha x + b) (chain.cu): one pass when fused,
+// else three passes through tmp. Arguments already validated.
+int launch_chain(const void* x, const void* b, void* y, void* tmp, long long rows, int cols,
+                 float alpha, int act, bool fused, cudaStream_t stream);
+
 // Unfused three-kernel path (naive.cu). Arguments already validated.
 int launch_naive(const AttnArgs& a, void* workspace, cudaStream_t stream);
 

@@ -70,6 +70,9 @@ def _load():
                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                            ctypes.c_void_p, i64p, ctypes.c_int64, f64p, f64p, ctypes.c_int]
+        lib.oracle_chain_bf16.restype = ctypes.c_int
+        lib.oracle_chain_bf16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                          ctypes.c_int, ctypes.c_double, ctypes.c_int, f64p]
         lib.oracle_probs_f64.restype = ctypes.c_int
         lib.oracle_probs_f64.argtypes = [f64p, f64p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_double, ctypes.c_int,
@@ -219,3 +222,23 @@ def probs_row(q: np.ndarray, k: np.ndarray, scale: float, causal: bool, i: int):
     if st != 0:
         raise RuntimeError(f"oracle_probs_f64 failed with status {st}")
     return p
+
+
+CHAIN_ACTS = {"relu": 0, "gelu": 1, "silu": 2}
+
+
+def chain(x, b, alpha: float, act: str):
+    """y = act(alpha * x + b) in double for bf16 torch tensors x [rows, cols]
+    and b [cols] (the elementwise chain); returns a float64 numpy array."""
+    lib = _load()
+    xa = _as_bf16_bits(x).reshape(-1)
+    ba = _as_bf16_bits(b).reshape(-1)
+    rows, cols = int(x.shape[0]), int(x.shape[1])
+    if ba.shape[0] != cols:
+        raise ValueError("one bias per column expected")
+    y = np.zeros((rows, cols), dtype=np.float64)
+    st = lib.oracle_chain_bf16(xa.ctypes.data, ba.ctypes.data, rows, cols, float(alpha),
+                               CHAIN_ACTS[act], y.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if st != 0:
+        raise RuntimeError(f"oracle_chain_bf16 failed with status {st}")
+    return y

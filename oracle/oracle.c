@@ -326,3 +326,27 @@ int oracle_probs_f64(const double *q, const double *k, int N, int d,
     softmax_row(p + j0, j1 - j0, &m, &l);
     return 0;
 }
+
+/* The elementwise chain of the anylearn.cc page ("multiply a tensor by a
+ * scalar, add a bias, apply an activation"): y[r, c] = act(alpha * x[r, c] +
+ * b[c]) for bf16 x [rows, cols] and b [cols], in double. act 0: max(z, 0);
+ * 1: z * (1 + erf(z / sqrt(2))) / 2 (GELU with the exact normal CDF);
+ * 2: z / (1 + exp(-z)) (SiLU). Returns 0, or -1 on bad arguments. */
+int oracle_chain_bf16(const uint16_t *x, const uint16_t *b, int64_t rows, int cols,
+                      double alpha, int act, double *y) {
+    if (!x || !b || !y || rows < 1 || cols < 1 || act < 0 || act > 2) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int c = 0; c < cols; ++c) {
+            double z = alpha * bf16_bits_to_double(x[r * cols + c]) + bf16_bits_to_double(b[c]);
+            double out;
+            if (act == 0)
+                out = z > 0.0 ? z : 0.0;
+            else if (act == 1)
+                out = 0.5 * z * (1.0 + erf(z / sqrt(2.0)));
+            else
+                out = z / (1.0 + exp(-z));
+            y[r * cols + c] = out;
+        }
+    }
+    return 0;
+}

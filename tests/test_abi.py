@@ -9,7 +9,8 @@ import exact_attention_125_b200 as ea
 from exact_attention_125_b200 import _build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "attn.h")
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
 
 
 @pytest.fixture(scope="module")
@@ -19,15 +20,18 @@ def L():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b((?:attn|chain)_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("attn_fwd", "attn_fwd_naive", "attn_fwd_naive_workspace_bytes",
-                 "attn_last_device_error", "attn_status_string"):
+                 "attn_last_device_error", "attn_status_string", "attn_fwd_kv", "attn_fwd_ext",
+                 "chain_fused", "chain_unfused"):
         assert want in names
 
 
@@ -152,3 +156,20 @@ def test_ext_workspace_counts_only_the_window():
     assert f(1, 2, 1, 1000, 64, 127, 2) == 2 * 2 * 64 * 4 + 2 * 2 * 4 + (256 - (2 * 2 * 64 * 4) % 256) % 256
     assert f(1, 2, 1, 1000, 64, -1, 8) == ea.abi.attn_fwd_kv_workspace_bytes(1, 2, 1, 1000, 64, 8)
     assert f(1, 2, 1, 1000, 64, -2, 8) == 0
+
+
+def test_chain_argument_errors(L):
+    f, u = ea.lib().chain_fused, ea.lib().chain_unfused
+    import ctypes
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_float,
+                                          ctypes.c_int, ctypes.c_void_p]
+    u.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_float,
+                                          ctypes.c_int, ctypes.c_void_p]
+    assert f(None, A, A, 4, 64, 1.0, 0, None) == -1
+    assert f(A, A, A, 4, 60, 1.0, 0, None) == -2          # cols not a multiple of 8
+    assert f(A, A, A, 0, 64, 1.0, 0, None) == -2
+    assert f(A + 8, A, A, 4, 64, 1.0, 0, None) == -4
+    assert f(A, A, A, 4, 64, float("nan"), 0, None) == -5
+    assert f(A, A, A, 4, 64, 1.0, 3, None) == -6
+    assert u(A, A, A, None, 4, 64, 1.0, 1, None) == -1
+    assert u(A, A, A, A + 4, 4, 64, 1.0, 1, None) == -4

@@ -331,3 +331,28 @@ def test_ext_bias_vanishes_at_the_own_position():
     o1, l1 = oracle.attention_ext(q, k, v, 0.5, True, 0, -1, None)
     o2, l2 = oracle.attention_ext(q, k, v, 0.5, True, 0, -1, [3.0])
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)  # |pos - pos| = 0
+
+
+# --------------------------------------------------------- elementwise chain
+def test_chain_closed_forms():
+    # x = 2, b = -1, alpha = 0.5 -> z = 0 everywhere; x = 4, alpha = 0.5, b = 0 -> z = 2
+    x = torch.tensor([[2.0, 4.0, -6.0, 1.0]], dtype=torch.bfloat16)
+    b = torch.tensor([-1.0, 0.0, 1.0, 0.0], dtype=torch.bfloat16)
+    z = np.array([0.0, 2.0, -2.0, 0.5])
+    np.testing.assert_array_equal(oracle.chain(x, b, 0.5, "relu")[0], np.maximum(z, 0))
+    g = oracle.chain(x, b, 0.5, "gelu")[0]
+    # z Phi(z): Phi(0) = 1/2, Phi(2) = 0.9772498680518208, Phi(-2) = 1 - Phi(2)
+    np.testing.assert_allclose(g, [0.0, 2 * 0.9772498680518208, -2 * (1 - 0.9772498680518208),
+                                   0.5 * 0.6914624612740131], rtol=1e-15, atol=0)
+    s = oracle.chain(x, b, 0.5, "silu")[0]
+    np.testing.assert_allclose(s, z / (1 + np.exp(-z)), rtol=1e-15, atol=0)
+
+
+@pytest.mark.parametrize("act", ["relu", "gelu", "silu"])
+def test_chain_matches_torch_float64(act):
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn((5, 16), generator=g).mul(3).to(torch.bfloat16)
+    b = torch.randn((16,), generator=g).to(torch.bfloat16)
+    z = 1.75 * x.double() + b.double()
+    ref = {"relu": torch.relu, "gelu": torch.nn.functional.gelu, "silu": torch.nn.functional.silu}[act](z)
+    np.testing.assert_allclose(oracle.chain(x, b, 1.75, act), ref.numpy(), rtol=1e-14, atol=1e-15)
