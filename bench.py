@@ -636,7 +636,7 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
 
 
 def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
-    """y = gelu(0.5 x + b) over a [65536, 8192] bf16 tensor (1 GiB, above L2),
+    """y = gelu_tanh(0.5 x + b) over a [65536, 8192] bf16 tensor (1 GiB, above L2),
     one fused kernel against three: achieved GB/s of each path's own traffic
     (fused: x read, y written; unfused: three reads and three writes) and the
     time ratio the page predicts to be about 3."""
@@ -650,8 +650,8 @@ def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
     tmp = torch.empty_like(x)
     stream = torch.cuda.current_stream(device)
     out = {}
-    for name, fn in (("fused", lambda: ea.chain_fused(x, b, y, 0.5, "gelu", stream)),
-                     ("unfused", lambda: ea.chain_unfused(x, b, y, tmp, 0.5, "gelu", stream))):
+    for name, fn in (("fused", lambda: ea.chain_fused(x, b, y, 0.5, "gelu_tanh", stream)),
+                     ("unfused", lambda: ea.chain_unfused(x, b, y, tmp, 0.5, "gelu_tanh", stream))):
         for _ in range(warmup):
             fn()
         torch.cuda.synchronize(device)
@@ -669,7 +669,7 @@ def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
                      "launches_per_step": 1 if name == "fused" else 3}
     del x, y, tmp
     torch.cuda.empty_cache()
-    return {"workload": f"gelu(0.5 x + b), x [{rows}, {cols}] bf16", "bound": "hbm",
+    return {"workload": f"gelu_tanh(0.5 x + b), x [{rows}, {cols}] bf16", "bound": "hbm",
             "hbm_peak_gbs": float(peaks["hbm_gbs"]), **out,
             "speedup_fused_over_unfused": out["unfused"]["ms_per_step"] / out["fused"]["ms_per_step"],
             "kernel": "chain_pass_kernel"}

@@ -309,7 +309,7 @@ def attn_fwd_ext(q, k, v, o=None, lse=None, scale=None, causal=False, window_lef
 
 
 # CHAIN_ACT_* of include/chain.h
-CHAIN_ACTS = {"relu": 0, "gelu": 1, "silu": 2}
+CHAIN_ACTS = {"relu": 0, "gelu": 1, "silu": 2, "gelu_tanh": 3}
 
 
 def _check_chain(x, b):

@@ -264,7 +264,7 @@ int validate_chain(const void* x, const void* b, const void* y, long long rows, 
   if (rows > (1ll << 62) / cols) return ATTN_ERR_SHAPE;
   if (!aligned(x, 16) || !aligned(b, 16) || !aligned(y, 16)) return ATTN_ERR_ALIGN;
   if (!std::isfinite(alpha)) return ATTN_ERR_SCALE;
-  if (act < CHAIN_ACT_RELU || act > CHAIN_ACT_SILU) return ATTN_ERR_CAUSAL;
+  if (act < CHAIN_ACT_RELU || act > CHAIN_ACT_GELU_TANH) return ATTN_ERR_CAUSAL;
   return ATTN_OK;
 }
 

@@ -15,7 +15,9 @@
  *     y[r, c] = act(alpha * x[r, c] + b[c])
  *
  * act: CHAIN_ACT_RELU max(z, 0); CHAIN_ACT_GELU z * Phi(z) with the exact
- * normal CDF Phi(z) = (1 + erf(z / sqrt 2)) / 2; CHAIN_ACT_SILU z / (1 + e^-z).
+ * normal CDF Phi(z) = (1 + erf(z / sqrt 2)) / 2; CHAIN_ACT_SILU z / (1 + e^-z);
+ * CHAIN_ACT_GELU_TANH z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))) / 2, the
+ * tanh form of GELU that GPT-2 uses.
  *
  * Conventions: x, b, y, tmp are bf16 DEVICE pointers owned by the caller,
  * 16-byte aligned, row-major contiguous; cols must be a multiple of 8 and
@@ -37,7 +39,7 @@
 extern "C" {
 #endif
 
-enum { CHAIN_ACT_RELU = 0, CHAIN_ACT_GELU = 1, CHAIN_ACT_SILU = 2 };
+enum { CHAIN_ACT_RELU = 0, CHAIN_ACT_GELU = 1, CHAIN_ACT_SILU = 2, CHAIN_ACT_GELU_TANH = 3 };
 
 /*
  * chain_fused - one kernel: reads x (and b), computes alpha * x + b and the

@@ -224,7 +224,7 @@ def probs_row(q: np.ndarray, k: np.ndarray, scale: float, causal: bool, i: int):
     return p
 
 
-CHAIN_ACTS = {"relu": 0, "gelu": 1, "silu": 2}
+CHAIN_ACTS = {"relu": 0, "gelu": 1, "silu": 2, "gelu_tanh": 3}
 
 
 def chain(x, b, alpha: float, act: str):

@@ -331,10 +331,11 @@ int oracle_probs_f64(const double *q, const double *k, int N, int d,
  * scalar, add a bias, apply an activation"): y[r, c] = act(alpha * x[r, c] +
  * b[c]) for bf16 x [rows, cols] and b [cols], in double. act 0: max(z, 0);
  * 1: z * (1 + erf(z / sqrt(2))) / 2 (GELU with the exact normal CDF);
- * 2: z / (1 + exp(-z)) (SiLU). Returns 0, or -1 on bad arguments. */
+ * 2: z / (1 + exp(-z)) (SiLU); 3: z * (1 + tanh(sqrt(2/pi) * (z + 0.044715 z^3))) / 2
+ * (GELU, tanh form). Returns 0, or -1 on bad arguments. */
 int oracle_chain_bf16(const uint16_t *x, const uint16_t *b, int64_t rows, int cols,
                       double alpha, int act, double *y) {
-    if (!x || !b || !y || rows < 1 || cols < 1 || act < 0 || act > 2) return -1;
+    if (!x || !b || !y || rows < 1 || cols < 1 || act < 0 || act > 3) return -1;
     for (int64_t r = 0; r < rows; ++r) {
         for (int c = 0; c < cols; ++c) {
             double z = alpha * bf16_bits_to_double(x[r * cols + c]) + bf16_bits_to_double(b[c]);
@@ -343,8 +344,10 @@ int oracle_chain_bf16(const uint16_t *x, const uint16_t *b, int64_t rows, int co
                 out = z > 0.0 ? z : 0.0;
             else if (act == 1)
                 out = 0.5 * z * (1.0 + erf(z / sqrt(2.0)));
-            else
+            else if (act == 2)
                 out = z / (1.0 + exp(-z));
+            else
+                out = 0.5 * z * (1.0 + tanh(sqrt(2.0 / acos(-1.0)) * (z + 0.044715 * z * z * z)));
             y[r * cols + c] = out;
         }
     }

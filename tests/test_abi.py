@@ -170,6 +170,7 @@ def test_chain_argument_errors(L):
     assert f(A, A, A, 0, 64, 1.0, 0, None) == -2
     assert f(A + 8, A, A, 4, 64, 1.0, 0, None) == -4
     assert f(A, A, A, 4, 64, float("nan"), 0, None) == -5
-    assert f(A, A, A, 4, 64, 1.0, 3, None) == -6
+    assert f(A, A, A, 4, 64, 1.0, 4, None) == -6
+    assert f(A, A, A, 4, 64, 1.0, -1, None) == -6
     assert u(A, A, A, None, 4, 64, 1.0, 1, None) == -1
     assert u(A, A, A, A + 4, 4, 64, 1.0, 1, None) == -4

@@ -6,7 +6,8 @@ once to bf16, so |y - y_ref| <= 2^-8 |y_ref| plus fp32 noise (erf/exp to a few
 fp32 ulps). The unfused path also rounds alpha * x and alpha * x + b to bf16
 between its kernels; each rounding moves z = alpha * x + b by at most
 2^-8 (|alpha x| + |z|) / 2 per step, and the activations' slopes are at most
-1.13 (GELU), 1.1 (SiLU), 1 (ReLU), so its bound adds 1.2 * 2^-8 (|alpha x| + |z|).
+1.13 (GELU, either form), 1.1 (SiLU), 1 (ReLU), so its bound adds
+1.2 * 2^-8 (|alpha x| + |z|).
 """
 import numpy as np
 import pytest
@@ -27,7 +28,7 @@ def _inputs(rows, cols, seed):
     return x, b
 
 
-@pytest.mark.parametrize("act", ["relu", "gelu", "silu"])
+@pytest.mark.parametrize("act", ["relu", "gelu", "silu", "gelu_tanh"])
 @pytest.mark.parametrize("rows,cols", [(1, 8), (3, 24), (257, 136), (1000, 1024)])
 def test_chain_fused_and_unfused(rows, cols, act):
     x, b = _inputs(rows, cols, rows * 7 + cols)
@@ -50,8 +51,8 @@ def test_chain_large_tensor_sampled():
     # sampled for the oracle
     x, b = _inputs(4096, 8192, 11)
     xg, bg = x.cuda(), b.cuda()
-    yf = ea.chain_fused(xg, bg, alpha=0.5, act="gelu").cpu()
+    yf = ea.chain_fused(xg, bg, alpha=0.5, act="gelu_tanh").cpu()
     rows = torch.tensor([0, 1, 777, 2048, 4095])
-    y_ref = oracle.chain(x[rows], b, 0.5, "gelu")
+    y_ref = oracle.chain(x[rows], b, 0.5, "gelu_tanh")
     ef = np.abs(yf[rows].double().numpy() - y_ref)
     assert (ef <= U * np.abs(y_ref) + 1e-6).all()

@@ -348,11 +348,12 @@ def test_chain_closed_forms():
     np.testing.assert_allclose(s, z / (1 + np.exp(-z)), rtol=1e-15, atol=0)
 
 
-@pytest.mark.parametrize("act", ["relu", "gelu", "silu"])
+@pytest.mark.parametrize("act", ["relu", "gelu", "silu", "gelu_tanh"])
 def test_chain_matches_torch_float64(act):
     g = torch.Generator().manual_seed(3)
     x = torch.randn((5, 16), generator=g).mul(3).to(torch.bfloat16)
     b = torch.randn((16,), generator=g).to(torch.bfloat16)
     z = 1.75 * x.double() + b.double()
-    ref = {"relu": torch.relu, "gelu": torch.nn.functional.gelu, "silu": torch.nn.functional.silu}[act](z)
+    ref = {"relu": torch.relu, "gelu": torch.nn.functional.gelu, "silu": torch.nn.functional.silu,
+           "gelu_tanh": lambda t: torch.nn.functional.gelu(t, approximate="tanh")}[act](z)
     np.testing.assert_allclose(oracle.chain(x, b, 1.75, act), ref.numpy(), rtol=1e-14, atol=1e-15)
