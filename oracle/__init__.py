@@ -70,6 +70,14 @@ def _load():
                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                            ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                            ctypes.c_void_p, i64p, ctypes.c_int64, f64p, f64p, ctypes.c_int]
+        lib.oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_attn_e4m3.restype = ctypes.c_int
+        lib.oracle_attn_e4m3.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                         ctypes.c_double, ctypes.c_int, i64p, ctypes.c_int64,
+                                         f64p, f64p, ctypes.c_int]
         lib.oracle_chain_bf16.restype = ctypes.c_int
         lib.oracle_chain_bf16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                           ctypes.c_int, ctypes.c_double, ctypes.c_int, f64p]
@@ -203,6 +211,43 @@ def attention_ext(q, k, v, scale: float, causal: bool, window_left: int = -1,
             rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
             o.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
             lse.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), int(nthreads))
+    if st != 0:
+        raise RuntimeError(f"oracle failed with status {st}")
+    return o, lse
+
+
+def e4m3_value(code: int) -> float:
+    """The value of one OCP FP8 E4M3 code (0..255), decoded by the oracle."""
+    return float(_load().oracle_e4m3_to_double(int(code)))
+
+
+def _as_e4m3_codes(t) -> np.ndarray:
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.float8_e4m3fn:
+        raise TypeError("FP8 entry expects torch.float8_e4m3fn tensors")
+    return t.detach().to("cpu").contiguous().view(torch.uint8).numpy()
+
+
+def attention_fp8(q, k, v, scale: float, q_descale: float, k_descale: float, v_descale: float,
+                  causal: bool, rows=None, nthreads: int = 0):
+    """Attention of the dequantized tensors q_descale * Q, k_descale * K,
+    v_descale * V, for E4M3 torch tensors [B, H, N, d]. Returns (o, lse)."""
+    lib = _load()
+    qa, ka, va = (_as_e4m3_codes(x) for x in (q, k, v))
+    if qa.ndim != 4 or ka.shape != qa.shape or va.shape != qa.shape:
+        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    B, H, N, d = (int(x) for x in qa.shape)
+    if rows is None:
+        rows = all_rows(B * H, N)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+    R = rows.shape[0]
+    o = np.zeros((R, d), dtype=np.float64)
+    lse = np.zeros((R,), dtype=np.float64)
+    st = lib.oracle_attn_e4m3(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, B, H, N, d,
+                              float(scale), float(q_descale), float(k_descale), float(v_descale),
+                              int(bool(causal)), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                              R, o.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                              lse.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), int(nthreads))
     if st != 0:
         raise RuntimeError(f"oracle failed with status {st}")
     return o, lse

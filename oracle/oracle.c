@@ -47,7 +47,7 @@
 #include <string.h>
 #include <unistd.h>
 
-enum { IN_BF16 = 0, IN_F64 = 1 };
+enum { IN_BF16 = 0, IN_F64 = 1, IN_E4M3 = 2 };
 
 /* bf16 is the upper half of an IEEE binary32; widening is exact. */
 static double bf16_bits_to_double(uint16_t bits) {
@@ -57,8 +57,27 @@ static double bf16_bits_to_double(uint16_t bits) {
     return (double)f;
 }
 
+/* OCP 8-bit floating point E4M3 (the "fn" variant: finite values and NaN
+ * only): sign bit, 4 exponent bits with bias 7, 3 mantissa bits. Exponent
+ * field 0 encodes subnormals m * 2^-9; exponent 15 with mantissa 7 is NaN
+ * (there is no infinity), so the largest value is 1.75 * 2^8 = 448. */
+double oracle_e4m3_to_double(uint8_t bits) {
+    int sign = (bits >> 7) & 1;
+    int e = (bits >> 3) & 0xF;
+    int m = bits & 0x7;
+    double mag;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m, -9);
+    else
+        mag = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
 static double load_elem(const void *base, int kind, int64_t idx) {
     if (kind == IN_F64) return ((const double *)base)[idx];
+    if (kind == IN_E4M3) return oracle_e4m3_to_double(((const uint8_t *)base)[idx]);
     return bf16_bits_to_double(((const uint16_t *)base)[idx]);
 }
 
@@ -311,6 +330,22 @@ int oracle_attn_ext_f64(const double *q, const double *k, const double *v, int B
                         int64_t nrows, double *o, double *lse, int nthreads) {
     return attend(q, k, v, IN_F64, B, H, Nq, Nk, d, scale, causal, wl, wr, slopes, rows,
                   nrows, o, lse, nthreads);
+}
+
+/* FP8 inputs: q, k, v hold E4M3 codes [B, H, N, d]; the values attended are
+ * q_descale * Q, k_descale * K, v_descale * V (decoded exactly, scaled in
+ * double), i.e. attention of the dequantized tensors. */
+int oracle_attn_e4m3(const uint8_t *q, const uint8_t *k, const uint8_t *v, int B, int H,
+                     int N, int d, double scale, double q_descale, double k_descale,
+                     double v_descale, int causal, const int64_t *rows, int64_t nrows,
+                     double *o, double *lse, int nthreads) {
+    if (!isfinite(q_descale) || !isfinite(k_descale) || !isfinite(v_descale)) return -3;
+    /* scores scale * (qd Q).(kd K) = (scale qd kd) Q.K; output vd * (P V) */
+    int st = attend(q, k, v, IN_E4M3, B, H, N, N, d, scale * q_descale * k_descale, causal, -1,
+                    -1, NULL, rows, nrows, o, lse, nthreads);
+    if (st != 0) return st;
+    for (int64_t r = 0; r < nrows * (int64_t)d; ++r) o[r] *= v_descale;
+    return 0;
 }
 
 /* The probability row p[0..N-1] of query i for a single head (q: [N, d],

@@ -357,3 +357,39 @@ def test_chain_matches_torch_float64(act):
     ref = {"relu": torch.relu, "gelu": torch.nn.functional.gelu, "silu": torch.nn.functional.silu,
            "gelu_tanh": lambda t: torch.nn.functional.gelu(t, approximate="tanh")}[act](z)
     np.testing.assert_allclose(oracle.chain(x, b, 1.75, act), ref.numpy(), rtol=1e-14, atol=1e-15)
+
+
+# -------------------------------------------------------------------- FP8
+def test_e4m3_decoder_table_values():
+    # sign, 4-bit exponent (bias 7), 3-bit mantissa; subnormals m * 2^-9; S.1111.111 = NaN
+    assert oracle.e4m3_value(0x00) == 0.0
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9
+    assert oracle.e4m3_value(0x08) == 2.0 ** -6
+    assert oracle.e4m3_value(0x38) == 1.0
+    assert oracle.e4m3_value(0x3C) == 1.5
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0xFE) == -448.0
+    assert oracle.e4m3_value(0x80) == 0.0 and np.signbit(oracle.e4m3_value(0x80))
+    assert np.isnan(oracle.e4m3_value(0x7F)) and np.isnan(oracle.e4m3_value(0xFF))
+
+
+def test_e4m3_decoder_matches_torch_for_all_codes():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_value(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert (np.isnan(got) == nan).all()
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_attention_is_attention_of_the_dequantized_tensors(causal):
+    g = torch.Generator().manual_seed(21)
+    q, k, v = (torch.randn((1, 2, 9, 8), generator=g).mul(40).to(torch.float8_e4m3fn) for _ in range(3))
+    qd, kd, vd = 0.02, 0.03, 0.5
+    o, lse = oracle.attention_fp8(q, k, v, 0.35, qd, kd, vd, causal)
+    deq = [t.to(torch.float64).numpy() * s for t, s in ((q, qd), (k, kd), (v, vd))]
+    o_ref, lse_ref = oracle.attention(*deq, 0.35, causal)
+    assert np.abs(o - o_ref).max() <= 1e-13 * max(1.0, np.abs(o_ref).max())
+    assert np.abs(lse - lse_ref).max() <= 1e-13 * max(1.0, np.abs(lse_ref).max())
