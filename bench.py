@@ -56,6 +56,7 @@ def parse_args(argv=None):
     p.add_argument("--no-kv", action="store_true", help="skip the split-KV inference lines")
     p.add_argument("--no-ext", action="store_true", help="skip the window / distance-bias lines")
     p.add_argument("--no-chain", action="store_true", help="skip the elementwise-chain line")
+    p.add_argument("--no-fp8", action="store_true", help="skip the FP8 line")
     p.add_argument("--kv-only", default=None, metavar="WORKLOAD",
                    help="run only the split-KV line of this inference workload (one GPU)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -367,6 +368,7 @@ def run_ours(args):
                                        for name in KV_BENCH_WORKLOADS]
     ext = None if args.no_ext else [ext_line(spec, device, peaks) for spec in EXT_BENCH]
     chain = None if args.no_chain else chain_line(device, peaks)
+    fp8 = None if args.no_fp8 else fp8_line(w, device, peaks)
 
     peak = float(peaks["bf16_tflops"])
     line = {
@@ -415,6 +417,9 @@ def run_ours(args):
         line["masks_and_bias"] = ext
     if chain is not None:
         line["elementwise_chain"] = chain
+    if fp8 is not None:
+        fp8["speedup_over_bf16_line"] = ms_step / fp8["ms_per_step"]
+        line["fp8"] = fp8
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, n, cores, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -673,6 +678,49 @@ def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
             "hbm_peak_gbs": float(peaks["hbm_gbs"]), **out,
             "speedup_fused_over_unfused": out["unfused"]["ms_per_step"] / out["fused"]["ms_per_step"],
             "kernel": "chain_pass_kernel"}
+
+
+def fp8_line(w, device, peaks, steps=10, warmup=3):
+    """attn_fwd_fp8 on the headline shape: N(0,1) Q, K, V quantised per tensor
+    to E4M3 on the device; TFLOP/s against the FP8 dense peak, taken as the
+    measured bf16 burst figure times the nominal FP8 / bf16 ratio of 2."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    from exact_attention_125_b200 import costs
+    from exact_attention_125_b200.inputs import quantize_e4m3
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    qkv = [quantize_e4m3(torch.randn(w.shape, device=device, generator=g)) for _ in range(3)]
+    (q8, qd), (k8, kd), (v8, vd) = qkv
+    o = torch.empty(w.shape, dtype=torch.bfloat16, device=device)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        ea.attn_fwd_fp8(q8, k8, v8, qd, kd, vd, o, lse, scale=w.scale, causal=w.causal,
+                        stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    if ea.last_device_error() != 0:
+        raise SystemExit("device watchdog fired in the FP8 line")
+    ms = start.elapsed_time(end) / steps
+    tf = costs.attn_flops(w.B, w.H, w.N, w.d, w.causal) / (ms * 1e-3) / 1e12
+    peak = 2.0 * float(peaks["bf16_tflops"])
+    del q8, k8, v8, qkv
+    torch.cuda.empty_cache()
+    return {"workload": w.name + " (E4M3 Q, K, V)", "ms_per_step": ms, "steps": steps,
+            "tflops": tf, "bound": "tensor", "peak_tflops": peak,
+            "peak_source": "2 x MEASURED_PEAKS.json bf16_tflops (nominal FP8 / bf16 ratio)",
+            "frac": tf / peak, "speedup_over_bf16_line": None,
+            "kernel": "fused_attn_fwd_kernel<128, false, true>"}
 
 
 def main(argv=None):

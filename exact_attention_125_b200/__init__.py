@@ -18,6 +18,7 @@ import threading
 __all__ = [
     "AttnError", "lib", "attn_fwd", "attn_fwd_kv", "kv_num_splits", "kv_workspace_bytes",
     "attn_fwd_ext", "ext_num_splits", "ext_workspace_bytes", "chain_fused", "chain_unfused",
+    "attn_fwd_fp8",
     "CHAIN_ACTS",
     "attn_fwd_naive", "naive_workspace_bytes",
     "last_device_error", "status_string", "selftest_wait_timeout", "abi",
@@ -61,6 +62,8 @@ def lib() -> ctypes.CDLL:
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.attn_fwd.restype = i
+        L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, f, f, f, i, vp]
+        L.attn_fwd_fp8.restype = i
         L.attn_fwd_kv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
         L.attn_fwd_kv.restype = i
         L.attn_fwd_kv_num_splits.argtypes = [i, i, i, i, i]
@@ -103,6 +106,12 @@ class abi:
     @staticmethod
     def attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream) -> int:
         return lib().attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream)
+
+    @staticmethod
+    def attn_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, q_descale, k_descale, v_descale, causal,
+                     stream) -> int:
+        return lib().attn_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, q_descale, k_descale,
+                                  v_descale, causal, stream)
 
     @staticmethod
     def attn_fwd_kv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, num_splits, ws, ws_bytes,
@@ -212,6 +221,32 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
                       B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o=None, lse=None, scale=None,
+                 causal=False, stream=None):
+    """FP8 forward: q, k, v are CUDA torch.float8_e4m3fn tensors [B, H, N, 128]
+    holding Q / q_descale etc. Returns (o bf16 [B, H, N, 128], lse fp32)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dtype != torch.float8_e4m3fn or t.dim() != 4 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous float8_e4m3fn [B, H, N, d] tensor")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+    B, H, N, d = (int(x) for x in q.shape)
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = abi.attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, H, N, d, scale, float(q_descale), float(k_descale), float(v_descale),
+                          int(bool(causal)), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8")
     return o, lse
 
 

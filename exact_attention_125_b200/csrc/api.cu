@@ -214,6 +214,19 @@ size_t attn_fwd_ext_workspace_bytes(int B, int H, int Nq, int Nk, int d, int win
   return ext_workspace_bytes(B, H, Nq, Nk, d, window_left, num_splits);
 }
 
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, float q_descale, float k_descale, float v_descale,
+                 int causal, attn_stream_t stream) {
+  int st = validate(q, k, v, o, lse, B, H, N, d, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (d != 128) return ATTN_ERR_HEADDIM;
+  for (float s : {q_descale, k_descale, v_descale})
+    if (!std::isfinite(s) || !(s > 0.0f)) return ATTN_ERR_SCALE;
+  if ((st = check_device()) != ATTN_OK) return st;
+  return attn::launch_fused_fp8(pack(q, k, v, o, lse, B, H, N, d, scale, causal), q_descale,
+                                k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t attn_fwd_naive_workspace_bytes(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return 0;
   const unsigned long long bh = static_cast<unsigned long long>(B) * H;

@@ -51,6 +51,7 @@
 
 #include "../../include/attn.h"
 #include "internal.h"
+#include "fp8.cuh"
 #include "sm100.cuh"
 #include "tmem_io.cuh"
 #include "watchdog.cuh"
@@ -86,12 +87,16 @@ __host__ __device__ constexpr bool poly_pair(int cc) {
   return kPolyPeriod > 0 && cc % (kPolyPeriod > 0 ? kPolyPeriod : 1) == kPolyPeriod - 1;
 }
 
-template <int D>
+// kF8: Q, K, V hold 8-bit E4M3 values (one byte each) instead of bf16.
+template <int D, bool kF8 = false>
 struct Cfg {
-  static constexpr int kTileBytes = kTileRows * D * 2;  // one 128 x D bf16 tile
-  static constexpr int kAtoms = D / 64;                 // 128-byte swizzle atoms per row
+  static constexpr int kElemBytes = kF8 ? 1 : 2;
+  static constexpr int kTileBytes = kTileRows * D * kElemBytes;  // one 128 x D tile
+  static constexpr int kAtoms = D * kElemBytes / 128;   // 128-byte swizzle atoms per row
   static constexpr int kAtomBytes = kTileRows * 128;    // 16 KiB
-  static constexpr int kStages = (D == 128) ? 4 : 8;  // tile slots of the ring
+  static constexpr int kStages = (kTileBytes == 32768) ? 4 : 8;  // tile slots of the ring
+  // elements of the reduced dimension per MMA instruction (32 bytes of it)
+  static constexpr int kMmaK = 32 / kElemBytes;
   static constexpr int kUnits = kStages / 2;           // (V, K) units in flight
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
@@ -112,6 +117,7 @@ struct FwdParams {
   void* o;
   float* lse;
   unsigned int* err;
+  float v_descale;  // FP8 path: O is scaled by it (1 otherwise)
   int N, BH, nqb, T;  // N = keys (and query rows of the square problem); T = KV tiles
   float scale_log2;
   int causal;
@@ -196,11 +202,11 @@ __device__ __forceinline__ void store_row_chunk(const FwdParams& p, bool partial
   }
 }
 
-template <int D, bool kKV>
+template <int D, bool kKV, bool kF8 = false>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, uint32_t bars,
                                              int bh, int q0, int n_kv, int g,
                                              const Watchdog& wd, int kv_lo) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kF8>;
   const int warp = threadIdx.x / 32;
   const int tid = threadIdx.x % 128;
   const uint32_t lane_base = static_cast<uint32_t>(32 * (warp % 4)) << 16;
@@ -314,7 +320,9 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     const uint64_t c2 = f2_pack(cs, cs);
     const uint64_t nm2 = f2_pack(neg_m, neg_m);
     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-    uint32_t pk[64];
+    // P in tensor memory: bf16 pairs (64 columns) or, for FP8, four E4M3
+    // values per column (32 columns; p <= 2^8 fits E4M3's range of 448)
+    uint32_t pk[kF8 ? 32 : 64];
 #pragma unroll
     for (int cc = 0; cc < 64; ++cc) {
       float x0, x1, p0, p1;
@@ -327,14 +335,26 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
         p1 = ex2_approx(x1);
       }
       acc[cc % 4] = f2_add(acc[cc % 4], f2_pack(p0, p1));
-      pk[cc] = pack_bf16x2(p0, p1);
+      if constexpr (kF8) {
+        const uint32_t h = pack_e4m3x2(p0, p1);
+        if (cc % 2 == 0)
+          pk[cc / 2] = h;
+        else
+          pk[cc / 2] |= h << 16;
+      } else {
+        pk[cc] = pack_bf16x2(p0, p1);
+      }
     }
     {
       float lo, hi;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
       l_run += lo + hi;
     }
-    tmem_st_x64(tS, pk);
+    if constexpr (kF8) {
+      tmem_st_x32(tS, pk);
+    } else {
+      tmem_st_x64(tS, pk);
+    }
     tmem_st_wait();
     tc_fence_before_sync();
     mbar_arrive(bar_p_ready);
@@ -344,8 +364,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     if (!ok) return;
     tc_fence_after_sync();
 
-    // Epilogue: O / l -> bf16, lse in natural log.
-    const float inv_l = 1.0f / l_run;
+    // Epilogue: O / l -> bf16 (times V's scale on the FP8 path), lse in natural log.
+    const float inv_l = kF8 ? p.v_descale / l_run : 1.0f / l_run;
     const bool valid = row < p.N;
     uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
                                            (static_cast<size_t>(bh) * p.N + row) * D);
@@ -456,11 +476,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
   }
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUtensorMap* tk,
                                               const CUtensorMap* tv, uint32_t base, uint32_t bars,
                                               int bh, int q0, int n_kv_b, const Watchdog& wd) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kF8>;
   const uint32_t sQ = base + C::kQOff;
   const uint32_t sRing = base + C::kRingOff;
   const uint32_t bar_q = bars;
@@ -509,10 +529,10 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
     drain_wait(bars + 8u * (1 + w % C::kUnits), (w / C::kUnits) & 1, wd);
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t bars, int na,
                                          int nb, const Watchdog& wd) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kF8>;
   const uint32_t sQ = base + C::kQOff;
   const uint32_t sRing = base + C::kRingOff;
   const uint32_t bar_q = bars;
@@ -520,8 +540,8 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   const uint32_t bar_p_ready0 = bar_s_full0 + 16u;
   const uint32_t bar_o_final0 = bar_s_full0 + 32u;
   const uint32_t bar_mma_done = bar_s_full0 + 48u;
-  constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-  constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+  constexpr uint32_t idesc_qk = kF8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t idesc_pv = kF8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
 
   // unit u (see producer_role): V_{u-1} in tile slot 2 (u % kUnits), K_u in the next one
   auto par_of = [](int u) { return static_cast<uint32_t>((u / C::kUnits) & 1); };
@@ -530,25 +550,38 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   auto v_slot = [](int u) { return 2 * (u % C::kUnits); };
   auto k_slot = [](int u) { return 2 * (u % C::kUnits) + 1; };
 
-  // S_g = Q_g K^T : A = Q tile (K-major), B = K tile (K-major), 16-deep steps.
+  // S_g = Q_g K^T : A = Q tile (K-major), B = K tile (K-major); each
+  // instruction reduces 32 bytes of d (16 bf16 or 32 E4M3 values), stepping
+  // through the 128-byte swizzle atoms of a row.
   auto issue_qk = [&](int g, int slot) {
     const uint32_t a0 = sQ + g * C::kTileBytes;
     const uint32_t b0 = sRing + slot * C::kTileBytes;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
+    for (int kk = 0; kk < D / C::kMmaK; ++kk) {
       const uint32_t off = (kk >> 2) * C::kAtomBytes + (kk & 3) * 32;
-      mma_ss(tmem + C::col_s(g), sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
-             idesc_qk, kk > 0 ? 1u : 0u);
+      if constexpr (kF8)
+        mma_ss_f8(tmem + C::col_s(g), sdesc_sw128(a0 + off, 16, 1024),
+                  sdesc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+      else
+        mma_ss(tmem + C::col_s(g), sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
+               idesc_qk, kk > 0 ? 1u : 0u);
     }
   };
-  // O_g += P_g V : A = P in tensor memory, B = V tile (MN-major), 16 keys per step.
+  // O_g += P_g V : A = P in tensor memory (8 columns per instruction: 16 bf16
+  // or 32 E4M3 keys), B = V tile (MN-major, rows of 128 bytes, one per key).
   auto issue_pv = [&](int g, int slot, bool accumulate) {
     const uint32_t b0 = sRing + slot * C::kTileBytes;
 #pragma unroll
-    for (int kk = 0; kk < kTileRows / 16; ++kk)
-      mma_ts(tmem + C::col_o(g), tmem + C::col_s(g) + kk * 8,
-             sdesc_sw128(b0 + kk * 2048, C::kAtomBytes, 1024), idesc_pv,
-             (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < kTileRows / C::kMmaK; ++kk) {
+      if constexpr (kF8)
+        mma_ts_f8(tmem + C::col_o(g), tmem + C::col_s(g) + kk * 8,
+                  sdesc_sw128(b0 + kk * C::kMmaK * 128, C::kAtomBytes, 1024), idesc_pv,
+                  (accumulate || kk > 0) ? 1u : 0u);
+      else
+        mma_ts(tmem + C::col_o(g), tmem + C::col_s(g) + kk * 8,
+               sdesc_sw128(b0 + kk * 2048, C::kAtomBytes, 1024), idesc_pv,
+               (accumulate || kk > 0) ? 1u : 0u);
+    }
   };
 
   bool ok = wait_one(bar_q, 0, wd) && wait_one(full_bar(0), par_of(0), wd);
@@ -776,12 +809,14 @@ __device__ __forceinline__ void mma_role_kv(uint32_t tmem, uint32_t base, uint32
 
 // kD: head dimension. kKV: the kv path (Nq query rows against N keys, the
 // KV range of each head split across CTAs); false: the square problem.
-template <int D, bool kKV>
+// kF8 (square problem only): E4M3 Q, K, V and P.
+template <int D, bool kKV, bool kF8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                           const __grid_constant__ CUtensorMap tmap_k,
                           const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
-  using C = Cfg<D>;
+  static_assert(!(kKV && kF8), "the FP8 path covers the square problem");
+  using C = Cfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // 128B swizzle wants 1024-byte alignment
@@ -845,14 +880,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
     const int g = warp / 4;
-    softmax_role<D, kKV>(p, tmem, bars, bh, q0, g == 0 ? na : nb, g, wd, kw.kv_lo);
+    softmax_role<D, kKV, kF8>(p, tmem, bars, bh, q0, g == 0 ? na : nb, g, wd, kw.kv_lo);
   } else {
     regs_decrease<kRegsOther>();
     if constexpr (!kKV) {
       if (warp == kProducerWarp) {
-        if (lane == 0) producer_role<D>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
+        if (lane == 0)
+          producer_role<D, kF8>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
       } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_role<D>(tmem, base, bars, na, nb, wd);
+        if (lane == 0) mma_role<D, kF8>(tmem, base, bars, na, nb, wd);
       }
     } else {
       const bool alt = p.alt != 0;
@@ -905,19 +941,22 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [B*H, N, d] bf16 viewed as a 3-D tensor (d innermost); box = 64 columns
-// (128 bytes, one swizzle atom) x 128 rows x 1 head; rows past N read as 0.
-bool encode_qkv_map(CUtensorMap* m, const void* ptr, int BH, int N, int d) {
+// [B*H, N, d] viewed as a 3-D tensor (d innermost) of bf16 (elem_bytes 2)
+// or E4M3 bytes (elem_bytes 1); box = 128 bytes of a row (one swizzle atom:
+// 64 bf16 or 128 E4M3) x 128 rows x 1 head; rows past N read as 0.
+bool encode_qkv_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int elem_bytes = 2) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTileRows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * elem_bytes};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes),
+                       static_cast<cuuint32_t>(kTileRows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = enc(m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -936,13 +975,17 @@ unsigned int* device_error_word() {
   return ptrs[dev];
 }
 
-template <int D>
-int launch_fused_d(const AttnArgs& a, cudaStream_t stream) {
-  using C = Cfg<D>;
+// kF8: Q, K, V are E4M3 with the given dequantisation scales (the scores get
+// q_descale * k_descale, O gets v_descale); otherwise bf16 and all scales 1.
+template <int D, bool kF8 = false>
+int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0f,
+                   float k_descale = 1.0f, float v_descale = 1.0f) {
+  using C = Cfg<D, kF8>;
   const int BH = a.B * a.H;
   CUtensorMap mq, mk, mv;
-  if (!encode_qkv_map(&mq, a.q, BH, a.N, D) || !encode_qkv_map(&mk, a.k, BH, a.N, D) ||
-      !encode_qkv_map(&mv, a.v, BH, a.N, D))
+  if (!encode_qkv_map(&mq, a.q, BH, a.N, D, C::kElemBytes) ||
+      !encode_qkv_map(&mk, a.k, BH, a.N, D, C::kElemBytes) ||
+      !encode_qkv_map(&mv, a.v, BH, a.N, D, C::kElemBytes))
     return ATTN_ERR_CUDA;
   unsigned int* err = device_error_word();
   if (!err) return ATTN_ERR_CUDA;
@@ -954,12 +997,14 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream) {
   p.BH = BH;
   p.nqb = (a.N + kBlockRows - 1) / kBlockRows;
   p.T = (a.N + kTileRows - 1) / kTileRows;
-  p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
+  p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * q_descale * k_descale *
+                                    1.4426950408889634);
+  p.v_descale = v_descale;
   p.causal = a.causal;
   p.wait_limit_ns = kWaitLimitNs;
   const long long grid = static_cast<long long>(p.nqb) * BH;
   if (grid > 0x7fffffffLL) return ATTN_ERR_SHAPE;
-  auto kernel = fused_attn_fwd_kernel<D, false>;
+  auto kernel = fused_attn_fwd_kernel<D, false, kF8>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
       cudaSuccess)
     return ATTN_ERR_CUDA;
@@ -1084,6 +1129,11 @@ int launch_fused_kv(const AttnKvArgs& a, const KvPlan& plan, void* workspace, cu
 
 int launch_fused(const AttnArgs& a, cudaStream_t stream) {
   return a.d == 128 ? launch_fused_d<128>(a, stream) : launch_fused_d<64>(a, stream);
+}
+
+int launch_fused_fp8(const AttnArgs& a, float q_descale, float k_descale, float v_descale,
+                     cudaStream_t stream) {
+  return launch_fused_d<128, true>(a, stream, q_descale, k_descale, v_descale);
 }
 
 int read_and_clear_device_error(cudaStream_t stream) {

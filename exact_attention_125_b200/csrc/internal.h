@@ -22,6 +22,11 @@ struct AttnArgs {
 // Fused tcgen05 path (fused_fwd.cu). Arguments already validated.
 int launch_fused(const AttnArgs& a, cudaStream_t stream);
 
+// FP8 variant (d = 128): q, k, v hold E4M3 bytes; the attended values are
+// q_descale * Q, k_descale * K, v_descale * V. Arguments already validated.
+int launch_fused_fp8(const AttnArgs& a, float q_descale, float k_descale, float v_descale,
+                     cudaStream_t stream);
+
 // kv path: Nq query rows against Nk keys per head.
 struct AttnKvArgs {
   const void* q;

@@ -186,3 +186,22 @@ def gather_rows(t: torch.Tensor, rows: np.ndarray) -> torch.Tensor:
     flat = t.reshape(B * H * N, *t.shape[3:])
     idx = torch.as_tensor(rows[:, 0] * N + rows[:, 1], dtype=torch.long, device=t.device)
     return flat.index_select(0, idx)
+
+
+def quantize_e4m3(t: torch.Tensor, target_amax: float = 448.0):
+    """Per-tensor E4M3 quantisation of a float tensor (any device): returns
+    (codes as torch.float8_e4m3fn, descale) with t ~= descale * codes; the
+    scale maps the tensor's largest magnitude to target_amax (round to
+    nearest, saturating)."""
+    amax = float(t.detach().abs().max().float().cpu())
+    descale = (amax / target_amax) if amax > 0 else 1.0
+    codes = (t.float() / descale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    return codes, descale
+
+
+def make_qkv_fp8(B: int, H: int, N: int, d: int, seed: int):
+    """make_qkv's N(0,1) draws, quantised per tensor to E4M3: returns
+    ((q8, k8, v8), (q_descale, k_descale, v_descale)) on the CPU."""
+    q, k, v = make_qkv(B, H, N, d, seed)
+    out = [quantize_e4m3(x) for x in (q, k, v)]
+    return tuple(c for c, _ in out), tuple(s for _, s in out)

@@ -88,6 +88,24 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              attn_stream_t stream);
 
 /*
+ * attn_fwd_fp8 - attn_fwd with 8-bit floating-point inputs, the low-precision
+ * step the anylearn.cc page credits FlashAttention-3 with (1.3 PFLOP/s in
+ * FP8 on an H100). q, k, v hold OCP E4M3 codes (1 byte each, the finite-only
+ * variant, largest value 448), [B, H, N, d] contiguous, 16-byte aligned; the
+ * values attended are q_descale * Q, k_descale * K and v_descale * V (per-
+ * tensor scales, finite and > 0, else ATTN_ERR_SCALE). d must be 128
+ * (ATTN_ERR_HEADDIM). o: bf16 [B, H, N, d]; lse: fp32 [B, H, N], as for
+ * attn_fwd. Both products run on the tensor cores in E4M3 with fp32
+ * accumulation: S = Q K^T from the E4M3 inputs, and P (the softmax weights
+ * 2^(x - m) <= 2^8, rounded to E4M3 to nearest) times V. The row sums and
+ * the log-sum-exp use the unrounded fp32 weights.
+ */
+int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
+                 float *lse, int B, int H, int N, int d, float scale,
+                 float q_descale, float k_descale, float v_descale, int causal,
+                 attn_stream_t stream);
+
+/*
  * attn_fwd_kv - fused attention of Nq query rows against Nk keys per head, the
  * long-context inference shape (a few new tokens against a long context:
  * pratikdhanave.com, "The Attention Bottleneck - and How FlashAttention Fixed
