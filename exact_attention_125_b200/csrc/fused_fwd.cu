@@ -109,6 +109,7 @@ struct Cfg {
   // warpgroups when they took alternate KV tiles of one query tile
   static constexpr int kXchOff = kMiscOff + 16;
   static constexpr int kSmemBytesKv = kXchOff + 256 * 2 * 4 + 1024;
+  static_assert(kSmemBytesKv <= 227 * 1024, "kv path exceeds the shared memory of a CTA");
   __host__ __device__ static constexpr uint32_t col_s(int g) { return g == 0 ? 0u : 128u; }
   __host__ __device__ static constexpr uint32_t col_o(int g) { return 256u + (g == 0 ? 0u : uint32_t(D)); }
 };
@@ -268,11 +269,33 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
       }
       if (p.slopes) {
         // linear distance bias: x = s * c - slope * log2(e) * |pos - key|
-        const float rel = static_cast<float>(row + p.offset - col0);
+        const float rel = static_cast<float>(row + p.offset - col0);  // pos - col0
+        const bool left = col0 + kTileRows - 1 <= row_start + p.offset;   // key <= pos everywhere
+        const bool right = col0 >= row_start + kTileRows - 1 + p.offset;  // key >= pos everywhere
+        if (left || right) {
+          // one side of every row's position: the bias is linear in the
+          // column, b(cc) = b0 + dk * cc, stepped in packed pairs
+          const float dk = left ? slope_l2 : -slope_l2;
+          const float b0 = -dk * rel;
+          uint64_t bpair = f2_pack(b0, b0 + dk);
+          const uint64_t step2 = f2_pack(2.0f * dk, 2.0f * dk);
+          const uint64_t c2b = f2_pack(c, c);
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc)
-          sr[cc] = __float_as_uint(
-              fmaf(__uint_as_float(sr[cc]), c, -slope_l2 * fabsf(rel - static_cast<float>(cc))));
+          for (int cc = 0; cc < 128; cc += 2) {
+            const uint64_t t = f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])),
+                                      c2b, bpair);
+            float t0, t1;
+            f2_unpack(t, t0, t1);
+            sr[cc] = __float_as_uint(t0);
+            sr[cc + 1] = __float_as_uint(t1);
+            bpair = f2_add(bpair, step2);
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 128; ++cc)
+            sr[cc] = __float_as_uint(
+                fmaf(__uint_as_float(sr[cc]), c, -slope_l2 * fabsf(rel - static_cast<float>(cc))));
+        }
         cs = 1.0f;
       }
     } else {
