@@ -218,6 +218,12 @@ def max_over_ranks(x: float, dist, device) -> float:
     return float(t.item())
 
 
+def aggregate_tflops(flops_per_rank_step: float, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processes its own copy of the workload
+    each step (weak scaling), timed as the slowest rank's device time."""
+    return flops_per_rank_step * world * steps / (ms_max * 1e-3) / 1e12
+
+
 def barrier(dist):
     if dist is not None:
         dist.barrier()
@@ -285,7 +291,7 @@ def run_reference(args):
     ms = statistics.median(s for _, s in per_step) * 1e3
     line = {
         "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s",
-        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
@@ -357,7 +363,7 @@ def run_ours(args):
     if ea.last_device_error() != 0:
         raise SystemExit("device watchdog fired in the timed region")
     ms_step = ms_total / args.steps
-    value = flops * world * args.steps / (ms_total * 1e-3) / 1e12
+    value = aggregate_tflops(flops, world, args.steps, ms_total)
     launch_tflops = flops / (ms_local / args.steps * 1e-3) / 1e12
     clock_info = clocks.summary()
 

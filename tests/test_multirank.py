@@ -1,0 +1,81 @@
+"""The N > 1 plumbing of bench.py on CPU: two ranks over gloo (spawned
+processes, 127.0.0.1 rendezvous). Each rank owns a different copy of the
+workload (weak scaling, no data-path collective); the only collectives are
+the barrier and the max over ranks of the timed duration; the reference arm
+prints from rank 0 alone."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    w_, r_, l_ = bench.dist_env()
+    dist = bench.init_dist(w_, "gloo")
+    bench.barrier(dist)
+    slowest = bench.max_over_ranks(10.0 + 5.0 * rank, dist, torch.device("cpu"))
+    from exact_attention_125_b200.inputs import WORKLOADS
+    q, k, v = bench._rank_inputs(WORKLOADS["single_head_128"], rank)
+    out.put((rank, w_, r_, slowest, float(q.float().sum()), float(k.float().sum())))
+    bench.barrier(dist)
+    dist.destroy_process_group()
+
+
+def test_two_ranks_share_only_timing():
+    ctx = mp.get_context("spawn")
+    out = ctx.SimpleQueue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(out.get() for _ in range(2))
+    assert [g[0] for g in got] == [0, 1] and all(g[1] == 2 for g in got)
+    assert all(g[3] == 15.0 for g in got)          # max over ranks seen by both
+    assert got[0][4] != got[1][4] and got[0][5] != got[1][5]  # each rank owns different inputs
+
+
+def test_aggregate_is_weak_scaling_over_the_slowest_rank():
+    one = bench.aggregate_tflops(4.0e12, 1, 10, 20.0)
+    assert one == pytest.approx(4.0e12 * 10 / 0.02 / 1e12)
+    # two ranks doing the same per-rank work in the same slowest time: twice the throughput
+    assert bench.aggregate_tflops(4.0e12, 2, 10, 20.0) == pytest.approx(2 * one)
+
+
+def test_reference_arm_prints_from_rank_zero_only():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1", MASTER_ADDR="127.0.0.1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_line_on_rank_zero():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "long_8192_causal"
