@@ -40,7 +40,7 @@ KV_PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_attn_fwd_kv_decode.tx
 # the sources that define the fused kernel; the ncu summary records their hash
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_125_b200", "csrc", f)
                   for f in ("fused_fwd.cu", "sm100.cuh", "tmem_io.cuh", "watchdog.cuh",
-                            "exp2_poly.cuh")]
+                            "exp2_poly.cuh", "fp8.cuh")]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
