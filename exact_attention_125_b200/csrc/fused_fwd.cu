@@ -26,7 +26,13 @@
 // (head, key range, query block); with Nq <= 128 its one query tile is shared
 // by both softmax warpgroups, which take alternate KV tiles and merge their
 // (O, m, l) at the end. Several ranges leave fp32 partial (O, lse) pairs that
-// lse_combine_kernel (combine.cu) merges.
+// lse_combine_kernel (combine.cu) merges. The same instantiation applies key
+// windows around each query's position (tiles outside every window are not
+// loaded) and an optional per-head linear distance bias.
+//
+// The FP8 instantiation (kF8 = true, square problem, d = 128) takes E4M3 Q,
+// K, V, runs both products as tcgen05 kind::f8f6f4 MMAs and stores P as four
+// E4M3 values per tensor-memory column (32 columns).
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_a [0,128), S_b [128,256),
 // O_a [256, 256+d), O_b [256+d, 256+2d). P (bf16, two per column) overwrites
