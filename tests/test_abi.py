@@ -174,3 +174,17 @@ def test_chain_argument_errors(L):
     assert f(A, A, A, 4, 64, 1.0, -1, None) == -6
     assert u(A, A, A, None, 4, 64, 1.0, 1, None) == -1
     assert u(A, A, A, A + 4, 4, 64, 1.0, 1, None) == -4
+
+
+def test_fp8_argument_errors(L):
+    f = ea.abi.attn_fwd_fp8
+    ok = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=128, scale=0.1, qd=0.01, kd=0.01,
+              vd=0.01, causal=1, stream=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"], a["d"],
+                 a["scale"], a["qd"], a["kd"], a["vd"], a["causal"], a["stream"])
+    assert call(d=64) == -3                      # FP8 path: d = 128 only
+    assert call(qd=0.0) == -5 and call(kd=float("inf")) == -5 and call(vd=-1.0) == -5
+    assert call(v=None) == -1 and call(k=A + 1) == -4 and call(N=0) == -2 and call(causal=5) == -6
