@@ -409,7 +409,7 @@ def run_ours(args):
             "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peaks_kind}, burst)",
             "traffic": profiled_traffic(),
             "algorithmic_bytes": costs.fused_bytes(w.B, w.H, w.N, w.d),
-            "kernel": "fused_attn_fwd_kernel<128, false>",
+            "kernel": "fused_attn_fwd_kernel<128, false, false>",
         },
         "clocks": {k: clock_info[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "e2e": e2e,
@@ -610,7 +610,7 @@ def split_kv_line(name, device, peaks, steps=10, warmup=3):
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
             "bound": "hbm", "traffic": profiled_kv_traffic(w),
-            "kernel": "fused_attn_fwd_kernel<128, true>" + (" + lse_combine_kernel<128>"
+            "kernel": "fused_attn_fwd_kernel<128, true, false>" + (" + lse_combine_kernel<128>"
                                                             if splits > 1 else ""),
             "tflops": flops / (ms * 1e-3) / 1e12,
             "launches_per_step": 2 if splits > 1 else 1,
@@ -670,7 +670,7 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
             "window_left": wl, "window_right": wr, "distance_bias": bias, "num_splits": splits,
             "ms_per_step": ms, "steps": steps, "tflops": tf, "bound": "tensor",
             "peak_tflops": float(peaks["bf16_tflops"]), "frac": tf / float(peaks["bf16_tflops"]),
-            "kernel": "fused_attn_fwd_kernel<128, true>"}
+            "kernel": "fused_attn_fwd_kernel<128, true, false>"}
 
 
 def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
