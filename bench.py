@@ -429,7 +429,9 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, n, cores, desc = cpu_oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": secs}
+                                "sample": desc, "seconds": secs, "rows_per_s": n / secs,
+                                "extrapolated_full_workload_s": flops / (tf * 1e12),
+                                "extrapolated": True}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
