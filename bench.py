@@ -352,13 +352,18 @@ def run_ours(args):
     with ClockSampler(local) as clocks:
         barrier(dist)
         torch.cuda.synchronize(device)
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
         start.record(stream)
-        for _ in range(args.steps):
+        for i in range(args.steps):
             step()
+            if i + 1 < args.steps:
+                marks[i].record(stream)
         end.record(stream)
         torch.cuda.synchronize(device)
         barrier(dist)
     ms_local = start.elapsed_time(end)
+    bounds = [start, *marks, end]
+    per_step = sorted(a.elapsed_time(b) for a, b in zip(bounds[:-1], bounds[1:]))
     ms_total = max_over_ranks(ms_local, dist, device)
     if ea.last_device_error() != 0:
         raise SystemExit("device watchdog fired in the timed region")
@@ -385,6 +390,8 @@ def run_ours(args):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
+        "ms_per_step_median_rank0": statistics.median(per_step),
+        "ms_per_step_best_rank0": per_step[0],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
