@@ -97,11 +97,14 @@ def _summary_fields(path):
     return fields
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary."""
+def profiled_traffic(workload: str = WORKLOAD):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary
+    (taken on long_8192_causal; None for any other workload)."""
     fields = _summary_fields(PROFILE_SUMMARY)
+    if not fields or fields.get("workload", WORKLOAD) != workload:
+        return None
     try:
-        return float(fields["dram_bytes_per_launch_full_workload"]) if fields else None
+        return float(fields["dram_bytes_per_launch_full_workload"])
     except (KeyError, ValueError):
         return None
 
@@ -414,7 +417,7 @@ def run_ours(args):
             "unit": "TFLOP/s",
             "frac": launch_tflops / peak,
             "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peaks_kind}, burst)",
-            "traffic": profiled_traffic(),
+            "traffic": profiled_traffic(w.name),
             "algorithmic_bytes": costs.fused_bytes(w.B, w.H, w.N, w.d),
             "kernel": "fused_attn_fwd_kernel<128, false, false>",
         },
