@@ -5,8 +5,17 @@ directory). This module only marshals arguments: every step of the attention
 computation runs in the library's CUDA kernels. There is no CPU fallback; if
 the library is missing, every call raises.
 
-The torch-facing helpers take CUDA bf16 tensors of shape [B, H, N, d] and
-allocate outputs with torch when none are given (the library never allocates).
+The torch-facing helpers take CUDA tensors (bf16 [B, H, N, d] for attention,
+E4M3 for the FP8 path, bf16 [rows, cols] for the elementwise chain) and
+allocate outputs and workspaces with torch when none are given (the library
+never allocates):
+
+  attn_fwd        fused forward, square problem (causal or not)
+  attn_fwd_kv     Nq queries against Nk keys, key range split across CTAs
+  attn_fwd_ext    attn_fwd_kv with key windows and a per-head distance bias
+  attn_fwd_fp8    fused forward on E4M3 inputs with per-tensor scales
+  attn_fwd_naive  the unfused three-kernel path (S and P through HBM)
+  chain_fused / chain_unfused   act(alpha x + b) in one kernel or three
 """
 from __future__ import annotations
 
