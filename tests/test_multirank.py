@@ -79,3 +79,27 @@ def test_reference_arm_line_on_rank_zero():
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["config"]["workload"] == "long_8192_causal"
+
+
+def test_profiled_traffic_is_gated_by_source_hash_and_workload(tmp_path, monkeypatch):
+    good = tmp_path / "good.txt"
+    good.write_text(f"# header\nkernel_source_sha256_16: {bench.source_hash()}\n"
+                    "workload: long_8192_causal\ndram_bytes_per_launch_full_workload: 123\n")
+    stale = tmp_path / "stale.txt"
+    stale.write_text("kernel_source_sha256_16: 0000000000000000\n"
+                     "dram_bytes_per_launch_full_workload: 123\n")
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(good))
+    assert bench.profiled_traffic("long_8192_causal") == 123.0
+    assert bench.profiled_traffic("decoder_2048_causal") is None
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(stale))
+    assert bench.profiled_traffic("long_8192_causal") is None
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(tmp_path / "missing.txt"))
+    assert bench.profiled_traffic("long_8192_causal") is None
+
+
+def test_bench_arguments_parse():
+    a = bench.parse_args(["--gpus", "2", "--steps", "3", "--warmup", "4", "--no-naive",
+                          "--no-kv", "--no-ext", "--no-chain", "--no-fp8"])
+    assert (a.gpus, a.steps, a.warmup, a.impl) == (2, 3, 4, "ours")
+    assert a.no_naive and a.no_kv and a.no_ext and a.no_chain and a.no_fp8
+    assert bench.parse_args(["--impl", "reference"]).impl == "reference"
