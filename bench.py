@@ -57,6 +57,8 @@ def parse_args(argv=None):
     p.add_argument("--no-ext", action="store_true", help="skip the window / distance-bias lines")
     p.add_argument("--no-chain", action="store_true", help="skip the elementwise-chain line")
     p.add_argument("--no-fp8", action="store_true", help="skip the FP8 line")
+    p.add_argument("--no-square", action="store_true",
+                   help="skip the other square workloads and the host-overhead line")
     p.add_argument("--kv-only", default=None, metavar="WORKLOAD",
                    help="run only the split-KV line of this inference workload (one GPU)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -383,6 +385,9 @@ def run_ours(args):
     ext = None if args.no_ext else [ext_line(spec, device, peaks) for spec in EXT_BENCH]
     chain = None if args.no_chain else chain_line(device, peaks)
     fp8 = None if args.no_fp8 else fp8_line(w, device, peaks)
+    square = None if args.no_square else [square_line(name, device, peaks)
+                                          for name in SQUARE_BENCH_WORKLOADS]
+    host = None if args.no_square else host_overhead_line(device)
 
     peak = float(peaks["bf16_tflops"])
     line = {
@@ -425,6 +430,9 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": args.steps,
     }
+    if square is not None:
+        line["square_workloads"] = square
+        line["host_overhead_per_call"] = host
     if naive is not None:
         line["naive"] = naive
     if split_kv is not None:
@@ -569,6 +577,93 @@ def naive_line(w, device, peaks, steps=2):
             "hbm_peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
             "tflops": costs.attn_flops(w.B, w.H, w.N, w.d, w.causal) / (ms * 1e-3) / 1e12,
             "head_group": group, "launches_per_step": 3 * (BH // group)}
+
+
+# the other square workloads (the parity tests' configurations), each timed by
+# itself in a sub-line of the JSON line
+SQUARE_BENCH_WORKLOADS = ("single_head_128", "bert_base_1024", "decoder_2048_causal",
+                          "stress_65536_causal")
+
+
+def square_line(name, device, peaks):
+    """attn_fwd on one square workload: median and best device time of single
+    launches (CUDA events around each), TFLOP/s and the fraction of the bf16
+    peak. Small workloads sit in L2 and are launch-latency bound; their step
+    count is raised so the timed region spans ~50 ms."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    from exact_attention_125_b200 import costs
+    from exact_attention_125_b200.inputs import WORKLOADS, make_workload
+    w = WORKLOADS[name]
+    q, k, v = (t.to(device) for t in make_workload(w))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    flops = costs.attn_flops(w.B, w.H, w.N, w.d, w.causal)
+
+    def step():
+        ea.attn_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    step()
+    torch.cuda.synchronize(device)
+    est = max(time.perf_counter() - t0, 1e-6)
+    steps = int(min(200, max(5, 0.05 / est)))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    if ea.last_device_error() != 0:
+        raise SystemExit(f"device watchdog fired on {name}")
+    ts = sorted(a.elapsed_time(b) for a, b in zip(ev[:-1], ev[1:]))
+    med = statistics.median(ts)
+    peak = float(peaks["bf16_tflops"])
+    qkv_bytes = 3 * q.numel() * q.element_size()
+    return {"workload": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "steps": steps, "ms_median": med, "ms_best": ts[0],
+            "tflops": flops / (med * 1e-3) / 1e12, "tflops_best": flops / (ts[0] * 1e-3) / 1e12,
+            "frac": flops / (med * 1e-3) / 1e12 / peak, "bound": "tensor",
+            "l2": "inputs larger than L2" if qkv_bytes > 126e6 else "inputs fit in L2",
+            "launches_per_step": 1}
+
+
+def host_overhead_line(device, n_calls=2000):
+    """Host time of one attn_fwd call through the C ABI (argument checks,
+    tensor-map encoding, launch), on the smallest workload with the stream
+    left to run: the median over calls of the CPU time each call takes."""
+    import torch
+
+    import exact_attention_125_b200 as ea
+    from exact_attention_125_b200.inputs import WORKLOADS, make_workload
+    w = WORKLOADS["single_head_128"]
+    q, k, v = (t.to(device) for t in make_workload(w))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
+    s = torch.cuda.current_stream(device).cuda_stream
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
+            w.N, w.d, w.scale, int(w.causal), s)
+    f = ea.abi.attn_fwd
+    for _ in range(20):
+        f(*args)
+    torch.cuda.synchronize(device)
+    ts = []
+    for i in range(n_calls):
+        t0 = time.perf_counter_ns()
+        f(*args)
+        ts.append(time.perf_counter_ns() - t0)
+        if i % 100 == 99:
+            torch.cuda.synchronize(device)
+    torch.cuda.synchronize(device)
+    ts.sort()
+    return {"workload": w.name, "calls": n_calls, "us_median": ts[len(ts) // 2] / 1e3,
+            "us_p10": ts[len(ts) // 10] / 1e3, "us_p90": ts[9 * len(ts) // 10] / 1e3,
+            "includes": "Python ctypes call, validation, three tensor-map encodings, launch"}
 
 
 KV_BENCH_WORKLOADS = ("decode_131072", "chunk_128x32768_causal")

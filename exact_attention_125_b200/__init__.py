@@ -30,7 +30,8 @@ __all__ = [
     "attn_fwd_fp8",
     "CHAIN_ACTS",
     "attn_fwd_naive", "naive_workspace_bytes",
-    "last_device_error", "status_string", "selftest_wait_timeout", "abi",
+    "last_device_error", "status_string", "selftest_wait_timeout", "set_wait_limit_ms",
+    "wait_limit_ms", "abi",
     "NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -105,6 +106,10 @@ def lib() -> ctypes.CDLL:
         L.attn_selftest_wait_timeout.restype = i
         L.attn_selftest_exp2.argtypes = [vp, vp, i, vp]
         L.attn_selftest_exp2.restype = i
+        L.attn_set_wait_limit_ms.argtypes = [i]
+        L.attn_set_wait_limit_ms.restype = i
+        L.attn_wait_limit_ms.argtypes = []
+        L.attn_wait_limit_ms.restype = i
         _lib = L
         return L
 
@@ -186,6 +191,14 @@ class abi:
     @staticmethod
     def attn_selftest_exp2(x, y, n, stream) -> int:
         return lib().attn_selftest_exp2(x, y, n, stream)
+
+    @staticmethod
+    def attn_set_wait_limit_ms(ms) -> int:
+        return lib().attn_set_wait_limit_ms(ms)
+
+    @staticmethod
+    def attn_wait_limit_ms() -> int:
+        return lib().attn_wait_limit_ms()
 
 
 def status_string(status: int) -> str:
@@ -422,3 +435,14 @@ def last_device_error(stream=None) -> int:
 
 def selftest_wait_timeout(limit_ms: int, stream=None) -> int:
     return abi.attn_selftest_wait_timeout(int(limit_ms), _stream_handle(stream))
+
+
+def set_wait_limit_ms(ms: int) -> None:
+    """Limit of every bounded wait in the kernels launched from now on."""
+    st = abi.attn_set_wait_limit_ms(int(ms))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_set_wait_limit_ms")
+
+
+def wait_limit_ms() -> int:
+    return abi.attn_wait_limit_ms()

@@ -24,7 +24,7 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4))
     return ATTN_ERR_ALIGN;
-  if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_SCALE;
+  if (!std::isfinite(scale)) return ATTN_ERR_SCALE;
   if (causal != 0 && causal != 1) return ATTN_ERR_CAUSAL;
   return ATTN_OK;
 }
@@ -89,7 +89,7 @@ int validate_kv(const void* q, const void* k, const void* v, const void* o, cons
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4))
     return ATTN_ERR_ALIGN;
-  if (!std::isfinite(scale) || !(scale > 0.0f)) return ATTN_ERR_SCALE;
+  if (!std::isfinite(scale)) return ATTN_ERR_SCALE;
   if (causal != 0 && causal != 1) return ATTN_ERR_CAUSAL;
   if (causal && Nq > Nk) return ATTN_ERR_SHAPE;
   return ATTN_OK;
@@ -307,6 +307,14 @@ int attn_last_device_error(attn_stream_t stream) {
   return attn::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream));
 }
 
+int attn_set_wait_limit_ms(int ms) {
+  if (ms < 1 || ms > 600000) return ATTN_ERR_SHAPE;
+  attn::set_wait_limit_ms(ms);
+  return ATTN_OK;
+}
+
+int attn_wait_limit_ms(void) { return attn::wait_limit_ms(); }
+
 int attn_selftest_wait_timeout(int limit_ms, attn_stream_t stream) {
   if (limit_ms < 1 || limit_ms > 5000) return ATTN_ERR_SHAPE;
   int st = check_device();
@@ -330,7 +338,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_SHAPE: return "ATTN_ERR_SHAPE: B, H or N out of range";
     case ATTN_ERR_HEADDIM: return "ATTN_ERR_HEADDIM: d must be 64 or 128";
     case ATTN_ERR_ALIGN: return "ATTN_ERR_ALIGN: pointer misaligned";
-    case ATTN_ERR_SCALE: return "ATTN_ERR_SCALE: scale must be finite and > 0";
+    case ATTN_ERR_SCALE: return "ATTN_ERR_SCALE: scale must be finite (FP8 descales finite and > 0)";
     case ATTN_ERR_CAUSAL: return "ATTN_ERR_CAUSAL: causal must be 0 or 1";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: workspace too small";
     case ATTN_ERR_LAUNCH: return "ATTN_ERR_LAUNCH: kernel launch failed";

@@ -52,10 +52,12 @@
 
 #include <cmath>
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "ctx_cache.h"
 #include "internal.h"
 #include "fp8.cuh"
 #include "sm100.cuh"
@@ -84,7 +86,8 @@ static_assert(128 * (2 * kRegsSoftmax + kRegsOther) == kThreads * kRegsAtLaunch,
               "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 256 while m lags
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Bounded-wait limit handed to every launch (attn_set_wait_limit_ms).
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 
 // Which of a row's 64 (even, odd) column pairs take the FMA-pipe exponential
 // (exp2_poly_pair) instead of the MUFU one; kPolyPeriod = 0 means none.
@@ -132,7 +135,12 @@ struct FwdParams {
   unsigned int* err;
   float v_descale;  // FP8 path: O is scaled by it (1 otherwise)
   int N, BH, nqb, T;  // N = keys (and query rows of the square problem); T = KV tiles
+  // |scale| * log2(e) (times the FP8 descales); 0 when scale is 0, which
+  // makes every allowed logit 0 (a uniform softmax over the allowed keys)
   float scale_log2;
+  // tcgen05 instruction-descriptor bit that negates A (Q) in S = Q K^T: set
+  // when scale < 0, so the softmax always multiplies by a positive factor
+  uint32_t qk_negate;
   int causal;
   uint64_t wait_limit_ns;
   // kv path only (Nq query rows against N keys, KV range split across CTAs)
@@ -215,8 +223,10 @@ __device__ __forceinline__ void store_row_chunk(const FwdParams& p, bool partial
   }
 }
 
+// ctl: shared address of the control barriers s_full[2], p_ready[2],
+// o_final[2] (consecutive).
 template <int D, bool kKV, bool kF8 = false>
-__device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, uint32_t bars,
+__device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, uint32_t ctl,
                                              int bh, int q0, int n_kv, int g,
                                              const Watchdog& wd, int kv_lo) {
   using C = Cfg<D, kF8>;
@@ -225,14 +235,17 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
   const uint32_t lane_base = static_cast<uint32_t>(32 * (warp % 4)) << 16;
   const uint32_t tS = tmem + lane_base + C::col_s(g);
   const uint32_t tO = tmem + lane_base + C::col_o(g);
-  const uint32_t bar_s_full = bars + 8u * (1 + 2 * C::kStages + g);
-  const uint32_t bar_p_ready = bars + 8u * (1 + 2 * C::kStages + 2 + g);
-  const uint32_t bar_o_final = bars + 8u * (1 + 2 * C::kStages + 4 + g);
+  const uint32_t bar_s_full = ctl + 8u * g;
+  const uint32_t bar_p_ready = ctl + 8u * (2 + g);
+  const uint32_t bar_o_final = ctl + 8u * (4 + g);
   // kv path with alternate KV tiles: both warpgroups hold the same query rows
   const bool alt = kKV && p.alt;
   const int row_start = alt ? q0 : q0 + kTileRows * g;
   const int row = row_start + tid;
-  const float c = p.scale_log2;
+  // scale 0: allowed logits are replaced by 0 and masked ones stay -inf, then
+  // scaled by 1 (scaling -inf by 0 would give NaN)
+  const bool zero_scale = p.scale_log2 == 0.0f;
+  const float c = zero_scale ? 1.0f : p.scale_log2;
   // kv path: this row's allowed keys [key_lo, key_hi] (causal limit, window,
   // key count); the tile's first row has the lowest key_hi and its last row
   // the highest key_lo, which decide whether a KV tile needs masking at all.
@@ -271,13 +284,13 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     float cs = c;  // multiplier from the values in sr to log2-domain logits
     if constexpr (kKV) {
       col0 = (kv_lo + (alt ? 2 * j + g : j)) * kTileRows;
-      need_mask = (col0 + kTileRows - 1 > tile_hi) || (col0 < tile_lo);
+      need_mask = (col0 + kTileRows - 1 > tile_hi) || (col0 < tile_lo) || zero_scale;
       if (need_mask) {
         const int lim_hi = key_hi - col0;
         const int lim_lo = key_lo - col0;
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc)
-          if (cc > lim_hi || cc < lim_lo) sr[cc] = 0xff800000u;  // -inf
+          sr[cc] = (cc > lim_hi || cc < lim_lo) ? 0xff800000u : (zero_scale ? 0u : sr[cc]);  // -inf
       }
       if (p.slopes) {
         // linear distance bias: x = s * c - slope * log2(e) * |pos - key|
@@ -312,13 +325,14 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
       }
     } else {
       col0 = j * kTileRows;
-      need_mask = (p.causal && col0 + kTileRows - 1 > row_start) || (col0 + kTileRows > p.N);
+      need_mask =
+          (p.causal && col0 + kTileRows - 1 > row_start) || (col0 + kTileRows > p.N) || zero_scale;
       if (need_mask) {
         int lim = p.N - 1 - col0;
         if (p.causal) lim = min(lim, row - col0);
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc)
-          if (cc > lim) sr[cc] = 0xff800000u;  // -inf
+          sr[cc] = cc > lim ? 0xff800000u : (zero_scale ? 0u : sr[cc]);  // -inf
       }
     }
 
@@ -434,7 +448,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     const size_t row_index =
         (partial ? static_cast<size_t>(kw.split) * p.BH + bh : static_cast<size_t>(bh)) * p.Nq + row;
     float* lse_dst = partial ? p.part_lse : p.lse;
-    const uint32_t bar_o_final0 = bars + 8u * (1 + 2 * C::kStages + 4);
+    const uint32_t bar_o_final0 = ctl + 8u * 4;
     if (!alt) {
       if (ok && n_kv > 0) ok = warp_wait(bar_o_final, 0, wd);
       if (!ok) return;
@@ -566,7 +580,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
 
 template <int D, bool kF8 = false>
 __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t bars, int na,
-                                         int nb, const Watchdog& wd) {
+                                         int nb, uint32_t qk_negate, const Watchdog& wd) {
   using C = Cfg<D, kF8>;
   const uint32_t sQ = base + C::kQOff;
   const uint32_t sRing = base + C::kRingOff;
@@ -575,7 +589,8 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   const uint32_t bar_p_ready0 = bar_s_full0 + 16u;
   const uint32_t bar_o_final0 = bar_s_full0 + 32u;
   const uint32_t bar_mma_done = bar_s_full0 + 48u;
-  constexpr uint32_t idesc_qk = kF8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+  const uint32_t idesc_qk =
+      (kF8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0)) | qk_negate;
   constexpr uint32_t idesc_pv = kF8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
 
   // unit u (see producer_role): V_{u-1} in tile slot 2 (u % kUnits), K_u in the next one
@@ -734,7 +749,8 @@ __device__ __forceinline__ void producer_role_kv(const CUtensorMap* tq, const CU
 // kv path MMA issuer; the unit layout is the one producer_role_kv loads.
 template <int D>
 __device__ __forceinline__ void mma_role_kv(uint32_t tmem, uint32_t base, uint32_t bars, int na,
-                                            int nb, bool alt, const Watchdog& wd) {
+                                            int nb, bool alt, uint32_t qk_negate,
+                                            const Watchdog& wd) {
   using C = Cfg<D>;
   const uint32_t sQ = base + C::kQOff;
   const uint32_t sRing = base + C::kRingOff;
@@ -743,7 +759,7 @@ __device__ __forceinline__ void mma_role_kv(uint32_t tmem, uint32_t base, uint32
   const uint32_t bar_p_ready0 = bar_s_full0 + 16u;
   const uint32_t bar_o_final0 = bar_s_full0 + 32u;
   const uint32_t bar_mma_done = bar_s_full0 + 48u;
-  constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+  const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0) | qk_negate;
   constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
 
   auto par_of = [](int u) { return static_cast<uint32_t>((u / C::kUnits) & 1); };
@@ -915,7 +931,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
     const int g = warp / 4;
-    softmax_role<D, kKV, kF8>(p, tmem, bars, bh, q0, g == 0 ? na : nb, g, wd, kw.kv_lo);
+    softmax_role<D, kKV, kF8>(p, tmem, bars + 8u * (1 + 2 * C::kStages), bh, q0,
+                              g == 0 ? na : nb, g, wd, kw.kv_lo);
   } else {
     regs_decrease<kRegsOther>();
     if constexpr (!kKV) {
@@ -923,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0)
           producer_role<D, kF8>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
       } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_role<D, kF8>(tmem, base, bars, na, nb, wd);
+        if (lane == 0) mma_role<D, kF8>(tmem, base, bars, na, nb, p.qk_negate, wd);
       }
     } else {
       const bool alt = p.alt != 0;
@@ -932,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           producer_role_kv<D>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, kw.kv_lo,
                               alt ? na + nb : max(na, nb), alt, p.nqb > 1, wd);
       } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_role_kv<D>(tmem, base, bars, na, nb, alt, wd);
+        if (lane == 0) mma_role_kv<D>(tmem, base, bars, na, nb, alt, p.qk_negate, wd);
       }
     }
   }
@@ -962,6 +979,38 @@ __global__ void wait_timeout_selftest_kernel(unsigned int* err, uint64_t limit_n
 
 // ------------------------------------------------------------------- host
 
+}  // namespace
+
+bool current_context_id(unsigned long long* id) {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  if (ctx == nullptr) {
+    // the runtime binds the device's primary context to this thread lazily
+    if (cudaFree(nullptr) != cudaSuccess || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+      return false;
+  }
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+namespace {
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -979,7 +1028,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // [B*H, N, d] viewed as a 3-D tensor (d innermost) of bf16 (elem_bytes 2)
 // or E4M3 bytes (elem_bytes 1); box = 128 bytes of a row (one swizzle atom:
 // 64 bf16 or 128 E4M3) x 128 rows x 1 head; rows past N read as 0.
-bool encode_qkv_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int elem_bytes = 2) {
+bool encode_qkv_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int elem_bytes = 2,
+                    int box_rows = kTileRows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
@@ -987,7 +1037,7 @@ bool encode_qkv_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int e
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * elem_bytes};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes),
-                       static_cast<cuuint32_t>(kTileRows), 1};
+                       static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                    3, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -996,18 +1046,41 @@ bool encode_qkv_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int e
   return r == CUDA_SUCCESS;
 }
 
+// Device address of g_device_error in the current context.
 unsigned int* device_error_word() {
-  static unsigned int* ptrs[64] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<unsigned int*>(p);
-  }
-  return ptrs[dev];
+  static CtxCache<unsigned int*> cache;
+  unsigned int* ptr = nullptr;
+  if (!cache.get(&ptr, [](unsigned int** out) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return false;
+        *out = static_cast<unsigned int*>(p);
+        return true;
+      }))
+    return nullptr;
+  return ptr;
+}
+
+// Once per (kernel, context): raise the kernel's dynamic shared-memory limit
+// and check the register allocation the in-kernel register split relies on
+// (the softmax warpgroups' setmaxnreg increase draws on exactly the launch
+// allocation, so any other count could make it wait forever; the build also
+// rejects such a binary). Later calls in the same context reuse the verdict.
+template <auto Kernel>
+int prepare_kernel(int smem_bytes) {
+  static CtxCache<int> cache;
+  int status = ATTN_ERR_CUDA;
+  if (!cache.get(&status, [smem_bytes](int* out) {
+        cudaFuncAttributes fa{};
+        if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem_bytes) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, Kernel) != cudaSuccess)
+          return false;  // not cached: a later call may succeed
+        *out = (fa.numRegs == kRegsAtLaunch && fa.maxThreadsPerBlock >= kThreads) ? ATTN_OK
+                                                                                  : ATTN_ERR_LAUNCH;
+        return true;
+      }))
+    return ATTN_ERR_CUDA;
+  return status;
 }
 
 // kF8: Q, K, V are E4M3 with the given dequantisation scales (the scores get
@@ -1032,22 +1105,18 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0
   p.BH = BH;
   p.nqb = (a.N + kBlockRows - 1) / kBlockRows;
   p.T = (a.N + kTileRows - 1) / kTileRows;
-  p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * q_descale * k_descale *
-                                    1.4426950408889634);
+  p.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(a.scale)) * q_descale *
+                                    k_descale * 1.4426950408889634);
+  p.qk_negate = a.scale < 0.0f ? kIdescNegateA : 0u;
   p.v_descale = v_descale;
   p.causal = a.causal;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   const long long grid = static_cast<long long>(p.nqb) * BH;
   if (grid > 0x7fffffffLL) return ATTN_ERR_SHAPE;
-  auto kernel = fused_attn_fwd_kernel<D, false, kF8>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-      cudaSuccess)
-    return ATTN_ERR_CUDA;
-  // The register split inside the kernel assumes this exact allocation.
-  cudaFuncAttributes fa{};
-  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (fa.numRegs != kRegsAtLaunch || fa.maxThreadsPerBlock < kThreads) return ATTN_ERR_LAUNCH;
-  kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+  const int prep = prepare_kernel<fused_attn_fwd_kernel<D, false, kF8>>(C::kSmemBytes);
+  if (prep != ATTN_OK) return prep;
+  fused_attn_fwd_kernel<D, false, kF8>
+      <<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -1072,9 +1141,10 @@ int launch_fused_kv_d(const AttnKvArgs& a, const KvPlan& plan, void* workspace,
   p.BH = BH;
   p.nqb = plan.nqb;
   p.T = plan.T;
-  p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
+  p.scale_log2 = static_cast<float>(std::fabs(static_cast<double>(a.scale)) * 1.4426950408889634);
+  p.qk_negate = a.scale < 0.0f ? kIdescNegateA : 0u;
   p.causal = a.causal;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   p.Nq = a.Nq;
   p.offset = a.Nk - a.Nq;
   p.nsplit = plan.nsplit;
@@ -1092,14 +1162,10 @@ int launch_fused_kv_d(const AttnKvArgs& a, const KvPlan& plan, void* workspace,
   }
   const long long grid = static_cast<long long>(plan.nqb) * plan.nsplit * BH;
   if (grid > 0x7fffffffLL) return ATTN_ERR_SHAPE;
-  auto kernel = fused_attn_fwd_kernel<D, true>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::kSmemBytesKv) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  cudaFuncAttributes fa{};
-  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (fa.numRegs != kRegsAtLaunch || fa.maxThreadsPerBlock < kThreads) return ATTN_ERR_LAUNCH;
-  kernel<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytesKv, stream>>>(mq, mk, mv, p);
+  const int prep = prepare_kernel<fused_attn_fwd_kernel<D, true>>(C::kSmemBytesKv);
+  if (prep != ATTN_OK) return prep;
+  fused_attn_fwd_kernel<D, true>
+      <<<static_cast<unsigned>(grid), kThreads, C::kSmemBytesKv, stream>>>(mq, mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   if (plan.nsplit > 1)
     return launch_lse_combine(p.part_o, p.part_lse, a.o, a.lse, BH * a.Nq, D, plan.nsplit, stream);
@@ -1169,6 +1235,14 @@ int launch_fused(const AttnArgs& a, cudaStream_t stream) {
 int launch_fused_fp8(const AttnArgs& a, float q_descale, float k_descale, float v_descale,
                      cudaStream_t stream) {
   return launch_fused_d<128, true>(a, stream, q_descale, k_descale, v_descale);
+}
+
+void set_wait_limit_ms(int ms) {
+  g_wait_limit_ns.store(static_cast<uint64_t>(ms) * 1000000ull, std::memory_order_relaxed);
+}
+
+int wait_limit_ms() {
+  return static_cast<int>(g_wait_limit_ns.load(std::memory_order_relaxed) / 1000000ull);
 }
 
 int read_and_clear_device_error(cudaStream_t stream) {

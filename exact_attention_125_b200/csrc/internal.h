@@ -81,6 +81,11 @@ int launch_naive(const AttnArgs& a, void* workspace, cudaStream_t stream);
 // the current device (naive.cu); nullptr if the lookup failed.
 void* noalloc_scratch_ptr();
 
+// Limit of every bounded wait in the fused kernels, for launches made from
+// now on (fused_fwd.cu); default 2000 ms.
+void set_wait_limit_ms(int ms);
+int wait_limit_ms();
+
 // Device error word of the current device (fused_fwd.cu).
 int read_and_clear_device_error(cudaStream_t stream);
 

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "ctx_cache.h"
 #include "internal.h"
 
 namespace attn {
@@ -404,19 +405,16 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SC
 
 // Device address of g_noalloc_scratch on the current device. In host code the
 // array's name is only a host-side stand-in, so the address is looked up with
-// cudaGetSymbolAddress once per device (with that device current) and cached.
+// cudaGetSymbolAddress, with the device current, once per CUDA context (a
+// context re-created after cudaDeviceReset gets a fresh lookup) and cached.
 void* noalloc_scratch_ptr() {
-  static void* ptrs[64] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    ptrs[dev] = p;
-  }
-  return ptrs[dev];
+  static CtxCache<void*> cache;
+  void* ptr = nullptr;
+  if (!cache.get(&ptr, [](void** out) {
+        return cudaGetSymbolAddress(out, g_noalloc_scratch) == cudaSuccess;
+      }))
+    return nullptr;
+  return ptr;
 }
 
 }  // namespace attn

@@ -188,6 +188,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, ui
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// Instruction-descriptor bit 13: negate A.
+constexpr uint32_t kIdescNegateA = 1u << 13;
+
 // Shared-memory matrix descriptor, 128-byte swizzle.
 //   bits 0-13 start>>4, 16-29 leading byte offset>>4, 32-45 stride byte
 //   offset>>4, 46-47 version (1 on sm_100), 61-63 layout (2 = 128B swizzle).

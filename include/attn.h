@@ -30,7 +30,10 @@
  * - d (head dimension) must be 64 or 128 (the page's "d is 64 or 128").
  * - B, H, N >= 1; B*H*N must fit in a signed 32-bit int.
  * - scale: the logit multiplier (1/sqrt(d) for standard attention), applied
- *   as given; must be finite and > 0.
+ *   as given; any finite value. scale = 0 gives the uniform softmax over the
+ *   allowed keys (o = their mean of v, lse = ln of their count); a negative
+ *   scale weights the keys with the lowest q . k highest. Non-finite scale:
+ *   ATTN_ERR_SCALE.
  * - causal: 0 (every key) or 1 (key j allowed for query i iff j <= i).
  * - Arithmetic: bf16 operands, fp32 accumulation, fp32 softmax; O is rounded
  *   to bf16 (round to nearest even).
@@ -61,7 +64,7 @@ enum {
     ATTN_ERR_SHAPE = -2,              /* B, H or N < 1, or B*H*N too large */
     ATTN_ERR_HEADDIM = -3,            /* d is not 64 or 128 */
     ATTN_ERR_ALIGN = -4,              /* a pointer breaks its alignment rule */
-    ATTN_ERR_SCALE = -5,              /* scale is not finite, or <= 0 */
+    ATTN_ERR_SCALE = -5,              /* scale not finite; FP8 descale not finite and > 0 */
     ATTN_ERR_CAUSAL = -6,             /* causal is not 0 or 1 */
     ATTN_ERR_WORKSPACE = -7,          /* naive path: workspace too small */
     ATTN_ERR_LAUNCH = -8,             /* the CUDA launch failed */
@@ -161,10 +164,10 @@ size_t attn_fwd_kv_workspace_bytes(int B, int H, int Nq, int Nk, int d,
 
 /*
  * attn_fwd_ext - attn_fwd_kv with the variants a fused library usually does
- * not cover (anylearn.cc, "Attention Is Memory-Bound, and Nobody Noticed for
- * Five Years": "a custom attention bias, an unusual masking pattern, a novel
- * position encoding" fall off the fast path), computed inside the same fused
- * kernel:
+ * not cover (the anylearn.cc page "Attention Is Memory-Bound, and Nobody
+ * Noticed for Five Years", on why the library matters, names bespoke biases,
+ * masks and position encodings as what leaves the fast path), computed inside
+ * the same fused kernel:
  *
  * - a key window around the query's sequence position pos = i + (Nk - Nq):
  *   key j is allowed iff pos - window_left <= j (when window_left >= 0) and
@@ -266,6 +269,19 @@ int attn_fwd_naive_noalloc(const void *q, const void *k, const void *v,
  * itself failed. Synchronises `stream` (the only entry point that does).
  */
 int attn_last_device_error(attn_stream_t stream);
+
+/*
+ * attn_set_wait_limit_ms - sets the limit, in milliseconds of the device's
+ * global timer, of every bounded wait inside the library's kernels, for
+ * launches made after the call (process-wide; default 2000). A wait that runs
+ * out makes its CTA give up as described under attn_last_device_error. Raise
+ * it where the GPU is time-sliced with other work for long stretches, so that
+ * a preempted CTA is not mistaken for a stuck one; lower it to fail faster.
+ * ms: 1 .. 600000, else ATTN_ERR_SHAPE. attn_wait_limit_ms returns the value
+ * in effect.
+ */
+int attn_set_wait_limit_ms(int ms);
+int attn_wait_limit_ms(void);
 
 /* attn_status_string - a static, human-readable name for a status code. */
 const char *attn_status_string(int status);

@@ -4,9 +4,9 @@
  *
  * The anylearn.cc page "Attention Is Memory-Bound, and Nobody Noticed for
  * Five Years" (the paragraphs on the technique underneath) gives the small
- * case of the fusion principle the attention kernel applies: multiply a
- * tensor by a scalar, add a bias, apply an activation. Three kernels read and
- * write the whole tensor three times; one fused kernel reads it once and
+ * case of the fusion principle the attention kernel applies: a chain of a
+ * scaling, a bias and an activation. Run as three kernels, it reads and
+ * writes the whole tensor three times; one fused kernel reads it once and
  * writes the result once, the intermediates staying in registers, and should
  * run about three times faster because the arithmetic was never the cost.
  *

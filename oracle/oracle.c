@@ -307,9 +307,9 @@ int oracle_attn_kv_f64(const double *q, const double *k, const double *v, int B,
                   nrows, o, lse, nthreads);
 }
 
-/* Masked and position-biased variants (the "custom attention bias, unusual
- * masking pattern, novel position encoding" cases that the anylearn.cc page
- * says fall off a fused library's fast path): keys limited to the window
+/* Masked and position-biased variants (the bespoke biases, masks and
+ * position encodings that, per the anylearn.cc page, a fused library's fast
+ * path does not cover): keys limited to the window
  * [pos - wl, pos + wr] (negative bound = unbounded) on top of the causal
  * rule, and, when slopes is not NULL, the score of key j for a query at
  * position pos lowered by slopes[h] * |pos - j| (a linear distance bias per

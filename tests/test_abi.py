@@ -62,8 +62,8 @@ def _fwd(**kw):
     (dict(B=0), -2), (dict(N=0), -2), (dict(H=-3), -2), (dict(B=65536, H=65536), -2),
     (dict(d=96), -3), (dict(d=256), -3),
     (dict(q=A + 8), -4), (dict(o=A + 2), -4), (dict(lse=A + 2), -4),
-    (dict(scale=float("nan")), -5), (dict(scale=float("inf")), -5), (dict(scale=0.0), -5),
-    (dict(scale=-0.5), -5),
+    (dict(scale=float("nan")), -5), (dict(scale=float("inf")), -5),
+    (dict(scale=float("-inf")), -5),
     (dict(causal=2), -6),
 ])
 def test_fused_argument_errors(L, kw, code):
@@ -80,6 +80,19 @@ def test_naive_argument_errors(L):
     assert f(A, A, A, A, A, 1, 1, 128, 64, 0.1, 0, A + 4, n, None) == -4
     assert f(A, A, A, A, A, 1, 1, 128, 64, 0.1, 0, A, n - 1, None) == -7
     assert f(A, A, A, A, A, 1, 1, 40000, 64, 0.1, 0, A, 1 << 40, None) == -2
+
+
+def test_wait_limit_is_settable(L):
+    assert ea.wait_limit_ms() == 2000
+    try:
+        ea.set_wait_limit_ms(250)
+        assert ea.wait_limit_ms() == 250
+        for bad in (0, -5, 600001):
+            with pytest.raises(ea.AttnError):
+                ea.set_wait_limit_ms(bad)
+        assert ea.wait_limit_ms() == 250
+    finally:
+        ea.set_wait_limit_ms(2000)
 
 
 def test_selftest_argument_range(L):
@@ -108,7 +121,7 @@ def _kv(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(k=None), -1), (dict(Nq=0), -2), (dict(Nk=0), -2), (dict(B=70000, H=70000), -2),
     (dict(Nq=5, Nk=4, causal=1), -2),           # causal needs Nq <= Nk
-    (dict(d=80), -3), (dict(v=A + 4), -4), (dict(scale=0.0), -5), (dict(causal=3), -6),
+    (dict(d=80), -3), (dict(v=A + 4), -4), (dict(scale=float("nan")), -5), (dict(causal=3), -6),
     (dict(splits=-1), -2), (dict(splits=257), -2),
     (dict(splits=4), -1),                        # a split workspace is required
     (dict(splits=4, ws=A + 16, ws_bytes=1 << 30), -4),   # 256-byte alignment

@@ -44,20 +44,34 @@ def _slopes(kind, H):
 
 @pytest.mark.parametrize("B,H,Nq,Nk,d,causal,wl,wr,kind,splits", CASES)
 def test_ext_all_rows(B, H, Nq, Nk, d, causal, wl, wr, kind, splits):
+    _ext_case(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale_of(d))
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.1])
+@pytest.mark.parametrize("B,H,Nq,Nk,d,causal,wl,wr,kind,splits", [
+    (1, 2, 300, 300, 128, True, 63, -1, "alibi", 1),
+    (1, 2, 100, 1100, 128, True, 300, -1, None, 4),
+    (1, 4, 1, 3000, 64, False, -1, -1, "alibi", 3),
+])
+def test_ext_zero_and_negative_scale(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale):
+    _ext_case(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale)
+
+
+def _ext_case(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale):
     q, k, v = make_q_kv(B, H, Nq, Nk, d, seed=Nq * 13 + Nk + wl + 7 * wr + d)
     slopes = _slopes(kind, H)
     qg, kg, vg = (t.to("cuda") for t in (q, k, v))
     sl = torch.tensor(slopes, dtype=torch.float32, device="cuda") if slopes else None
     o = torch.full((B, H, Nq, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((B, H, Nq), float("nan"), dtype=torch.float32, device="cuda")
-    ea.attn_fwd_ext(qg, kg, vg, o, lse, scale=scale_of(d), causal=causal, window_left=wl,
+    ea.attn_fwd_ext(qg, kg, vg, o, lse, scale=scale, causal=causal, window_left=wl,
                     window_right=wr, alibi_slopes=sl, num_splits=splits)
     torch.cuda.synchronize()
     assert ea.last_device_error() == 0
     rows = oracle.all_rows(B * H, Nq)
     # the oracle gets the fp32 slopes the kernel uses, widened exactly
     sl64 = [float(np.float32(x)) for x in slopes] if slopes else None
-    o_ref, lse_ref = oracle.attention_ext(q, k, v, scale_of(d), causal, wl, wr, sl64, rows=rows)
+    o_ref, lse_ref = oracle.attention_ext(q, k, v, scale, causal, wl, wr, sl64, rows=rows)
     o_rows = gather_rows(o.cpu(), rows)
     lse_rows = gather_rows(lse.cpu().unsqueeze(-1), rows).squeeze(-1)
     empty = np.isneginf(lse_ref)
@@ -67,7 +81,7 @@ def test_ext_all_rows(B, H, Nq, Nk, d, causal, wl, wr, kind, splits):
     keep = ~empty
     e = compare(o_rows[torch.as_tensor(keep)], lse_rows[torch.as_tensor(keep)], o_ref[keep],
                 lse_ref[keep])
-    assert_within(e, f"{(B, H, Nq, Nk, d, causal, wl, wr, kind, splits)}")
+    assert_within(e, f"{(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale)}")
 
 
 def test_ext_without_options_matches_attn_fwd_kv_bit_for_bit():

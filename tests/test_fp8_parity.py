@@ -65,6 +65,15 @@ def test_fp8_small_all_rows(B, H, N, causal):
     _check(q8, k8, v8, ds, 128 ** -0.5, causal, oracle.all_rows(B * H, N), o, lse, (B, H, N, causal))
 
 
+@pytest.mark.parametrize("scale", [0.0, -(128 ** -0.5)])
+def test_fp8_zero_and_negative_scale(scale):
+    (q8, k8, v8), ds = make_qkv_fp8(1, 2, 300, 128, seed=71)
+    o, lse = ea.attn_fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), *ds, scale=scale, causal=True)
+    torch.cuda.synchronize()
+    assert ea.last_device_error() == 0
+    _check(q8, k8, v8, ds, scale, True, oracle.all_rows(2, 300), o, lse, f"scale {scale}")
+
+
 def test_fp8_long_sampled():
     B, H, N = 1, 4, 8192
     (q8, k8, v8), ds = make_qkv_fp8(B, H, N, 128, seed=99)

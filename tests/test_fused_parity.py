@@ -30,6 +30,11 @@ SMALL = [
     (2, 3, 384, 128, False),
     (1, 2, 640, 64, True),
     (1, 1, 1000, 64, False),
+    # several 256-row blocks with a ragged last one
+    (1, 2, 1300, 128, True),
+    (2, 1, 1536, 128, False),
+    (1, 1, 2049, 128, True),
+    (1, 1, 600, 128, False),
 ]
 
 
@@ -49,7 +54,7 @@ def test_small_shapes_all_rows(B, H, N, d, causal):
     check_against_oracle(q, k, v, o, lse, scale_of(d), causal, what=f"{(B, H, N, d, causal)}")
 
 
-@pytest.mark.parametrize("name", ["single_head_128", "bert_base_1024"])
+@pytest.mark.parametrize("name", ["single_head_128", "bert_base_1024", "decoder_2048_causal"])
 def test_workloads_all_rows(name):
     w = WORKLOADS[name]
     q, k, v = make_workload(w)
@@ -57,8 +62,7 @@ def test_workloads_all_rows(name):
     check_against_oracle(q, k, v, o, lse, w.scale, w.causal, what=name)
 
 
-@pytest.mark.parametrize("name", ["decoder_2048_causal", "long_8192_causal",
-                                  "stress_65536_causal"])
+@pytest.mark.parametrize("name", ["long_8192_causal", "stress_65536_causal"])
 def test_workloads_sampled_rows(name):
     w = WORKLOADS[name]
     q, k, v = make_workload(w)
@@ -121,3 +125,21 @@ def test_outputs_do_not_depend_on_stale_memory():
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, l2)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, -1.0])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_zero_and_negative_scale(d, causal, scale):
+    # any finite scale is accepted; a negative one favours the smallest q.k
+    q, k, v = make_qkv(1, 2, 333, d, seed=31 + d + int(causal))
+    o, lse = _run(q, k, v, scale, causal)
+    check_against_oracle(q, k, v, o, lse, scale, causal, what=f"scale {scale}, d {d}")
+    if scale == 0.0:
+        # closed form: the mean of the allowed values, lse = ln |allowed keys|
+        n = torch.arange(1, 334, dtype=torch.float64) if causal else torch.full((333,), 333.0,
+                                                                                 dtype=torch.float64)
+        vd = v.double()
+        mean = (vd.cumsum(2) / n[:, None]) if causal else vd.mean(2, keepdim=True).expand_as(vd)
+        assert (o.cpu().double() - mean).abs().max().item() <= 2e-2
+        assert (lse.cpu().double() - n.log()).abs().max().item() <= 1e-3 * np.log(333.0)

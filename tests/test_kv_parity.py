@@ -70,6 +70,19 @@ def test_small_shapes_all_rows(B, H, Nq, Nk, d, causal, splits):
     _check(q, k, v, o, lse, scale_of(d), causal, rows, f"{(B, H, Nq, Nk, d, causal, splits)}")
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.09])
+@pytest.mark.parametrize("B,H,Nq,Nk,d,causal,splits", [
+    (1, 2, 1, 1000, 128, False, 3),
+    (1, 2, 100, 1100, 128, True, 9),
+    (1, 2, 300, 2000, 64, False, 3),
+])
+def test_zero_and_negative_scale(B, H, Nq, Nk, d, causal, splits, scale):
+    q, k, v = make_q_kv(B, H, Nq, Nk, d, seed=Nq * 31 + Nk + d + 5)
+    o, lse = _run(q, k, v, scale, causal, splits)
+    rows = oracle.all_rows(B * H, Nq)
+    _check(q, k, v, o, lse, scale, causal, rows, f"{(B, H, Nq, Nk, d, causal, splits, scale)}")
+
+
 def test_split_count_does_not_change_the_result_beyond_rounding():
     # every split count computes the same function; results differ only by
     # fp32 rounding order and the bf16 rounding of O

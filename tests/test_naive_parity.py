@@ -35,6 +35,14 @@ def test_small_shapes(B, H, N, d, causal):
     check_naive_against_oracle(q, k, v, o, lse, scale_of(d), causal, what=f"naive {(B, H, N, d)}")
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.125])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_and_negative_scale(scale, causal):
+    q, k, v = make_qkv(1, 2, 300, 128, seed=41 + int(causal))
+    o, lse = _run(q, k, v, scale, causal)
+    check_naive_against_oracle(q, k, v, o, lse, scale, causal, what=f"naive scale {scale}")
+
+
 def test_bert_base_all_rows():
     w = WORKLOADS["bert_base_1024"]
     q, k, v = make_workload(w)
