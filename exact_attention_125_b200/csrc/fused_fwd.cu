@@ -86,20 +86,25 @@ static_assert(128 * (2 * kRegsSoftmax + kRegsOther) == kThreads * kRegsAtLaunch,
               "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 256 while m lags
+// Largest overestimate (log2 units) of a tile's maximum logit allowed when a
+// linear distance bias is bounded instead of applied before the maximum: the
+// largest weight of the tile is then still >= 2^-96, far from fp32 underflow.
+constexpr float kBiasBoundSlack = 96.0f;
 // Bounded-wait limit handed to every launch (attn_set_wait_limit_ms).
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 
 // Which of a row's 64 (even, odd) column pairs take the FMA-pipe exponential
-// (exp2_poly_pair) instead of the MUFU one; kPolyPeriod = 0 means none.
-constexpr int kPolyPeriod = 4;
-// FP8: the E4M3 MMAs take half the bf16 time, so the softmax is the longer leg
-// by far and the FMA pipe has room for one pair in three (measured: 1/3 beats
-// 1/4 by 4 % and 1/2 is slower than both).
+// (exp2_poly_pair) instead of the MUFU one. bf16: three pairs in eight (2, 5
+// and 7 of every eight), which took ~14 % off a tile's softmax arithmetic
+// against one in four, with the row sum moved after the P hand-off. FP8: the
+// E4M3 MMAs take half the bf16 time, so the softmax is the longer leg by far
+// and the FMA pipe has room for one pair in three (measured: 1/3 beats 1/4 by
+// 4 % and 1/2 is slower than both).
 constexpr int kPolyPeriodF8 = 3;
 template <bool kF8>
 __host__ __device__ constexpr bool poly_pair(int cc) {
-  constexpr int P = kF8 ? kPolyPeriodF8 : kPolyPeriod;
-  return P > 0 && cc % (P > 0 ? P : 1) == P - 1;
+  if constexpr (kF8) return cc % kPolyPeriodF8 == kPolyPeriodF8 - 1;
+  return (cc % 8) == 2 || (cc % 8) == 5 || (cc % 8) == 7;
 }
 
 // kF8: Q, K, V hold 8-bit E4M3 values (one byte each) instead of bf16.
@@ -282,6 +287,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     bool need_mask;
     int col0;
     float cs = c;  // multiplier from the values in sr to log2-domain logits
+    // kv path, distance bias on a tile wholly on one side of every row's
+    // position: b(cc) = bias_b0 + bias_dk * cc (log2 units), applied in the
+    // exponent rather than to sr
+    bool bias_linear = false;
+    float bias_b0 = 0.0f, bias_dk = 0.0f;
     if constexpr (kKV) {
       col0 = (kv_lo + (alt ? 2 * j + g : j)) * kTileRows;
       need_mask = (col0 + kTileRows - 1 > tile_hi) || (col0 < tile_lo) || zero_scale;
@@ -297,31 +307,21 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
         const float rel = static_cast<float>(row + p.offset - col0);  // pos - col0
         const bool left = col0 + kTileRows - 1 <= row_start + p.offset;   // key <= pos everywhere
         const bool right = col0 >= row_start + kTileRows - 1 + p.offset;  // key >= pos everywhere
-        if (left || right) {
-          // one side of every row's position: the bias is linear in the
-          // column, b(cc) = b0 + dk * cc, stepped in packed pairs
-          const float dk = left ? slope_l2 : -slope_l2;
-          const float b0 = -dk * rel;
-          uint64_t bpair = f2_pack(b0, b0 + dk);
-          const uint64_t step2 = f2_pack(2.0f * dk, 2.0f * dk);
-          const uint64_t c2b = f2_pack(c, c);
-#pragma unroll
-          for (int cc = 0; cc < 128; cc += 2) {
-            const uint64_t t = f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])),
-                                      c2b, bpair);
-            float t0, t1;
-            f2_unpack(t, t0, t1);
-            sr[cc] = __float_as_uint(t0);
-            sr[cc + 1] = __float_as_uint(t1);
-            bpair = f2_add(bpair, step2);
-          }
+        if ((left || right) && slope_l2 * (kTileRows - 1) <= kBiasBoundSlack) {
+          // One side of every row's position: the bias is linear in the
+          // column, b(cc) = b0 + dk * cc. The scores stay unbiased here; the
+          // row maximum is bounded by max(s) * c + max(b) and the bias enters
+          // the exponent's FMA (below), one packed add per pair.
+          bias_dk = left ? slope_l2 : -slope_l2;
+          bias_b0 = -bias_dk * rel;
+          bias_linear = true;
         } else {
 #pragma unroll
           for (int cc = 0; cc < 128; ++cc)
             sr[cc] = __float_as_uint(
                 fmaf(__uint_as_float(sr[cc]), c, -slope_l2 * fabsf(rel - static_cast<float>(cc))));
+          cs = 1.0f;  // sr now holds the biased log2-domain logits
         }
-        cs = 1.0f;
       }
     } else {
       col0 = j * kTileRows;
@@ -344,7 +344,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
       mx[(cc / 2) % 8] = fmax3(mx[(cc / 2) % 8], __uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1]));
     const float rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
                              fmaxf(mx[6], mx[7]));
-    const float m_tile = rmax * cs;
+    // with a linear bias left out of sr, rmax * c + max(b) bounds the tile's
+    // largest logit from above: p = 2^(x - m) <= 1 stays true when m is
+    // raised to it, and the result is the exact softmax whatever m is
+    const float m_tile =
+        bias_linear ? fmaf(rmax, cs, fmaxf(bias_b0, fmaf(bias_dk, kTileRows - 1, bias_b0))) : rmax * cs;
     const bool raise = m_tile > m_run + kRescaleThreshold;
     const float m_new = raise ? m_tile : m_run;
     const float alpha = raise ? ex2_approx(m_run - m_new) : 1.0f;
@@ -365,9 +369,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
 
     // p = 2^(s * c - m) for the 64 (even, odd) column pairs: scaling and
     // summing in packed f32x2 form; most exponentials on the MUFU (ex2), the
-    // pairs poly_pair picks on the FMA pipe (exp2_poly_pair).
+    // pairs poly_pair picks on the FMA pipe (exp2_poly_pair). A linear bias
+    // rides in the addend: (b(cc) - m, b(cc + 1) - m), stepped by 2 dk.
     const uint64_t c2 = f2_pack(cs, cs);
-    const uint64_t nm2 = f2_pack(neg_m, neg_m);
+    uint64_t nm2 = bias_linear ? f2_pack(bias_b0 + neg_m, bias_b0 + bias_dk + neg_m)
+                               : f2_pack(neg_m, neg_m);
+    const uint64_t bias_step2 = f2_pack(2.0f * bias_dk, 2.0f * bias_dk);
     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
     // P in tensor memory: bf16 pairs (64 columns) or, for FP8, four E4M3
     // values per column (32 columns; p <= 2^8 fits E4M3's range of 448)
@@ -377,13 +384,15 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
       float x0, x1, p0, p1;
       f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1])), c2, nm2),
                 x0, x1);
+      if (bias_linear) nm2 = f2_add(nm2, bias_step2);
       if (poly_pair<kF8>(cc)) {
         exp2_poly_pair(x0, x1, p0, p1);
       } else {
         p0 = ex2_approx(x0);
         p1 = ex2_approx(x1);
       }
-      acc[cc % 4] = f2_add(acc[cc % 4], f2_pack(p0, p1));
+      sr[2 * cc] = __float_as_uint(p0);
+      sr[2 * cc + 1] = __float_as_uint(p1);
       if constexpr (kF8) {
         const uint32_t h = pack_e4m3x2(p0, p1);
         if (cc % 2 == 0)
@@ -394,11 +403,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
         pk[cc] = pack_bf16x2(p0, p1);
       }
     }
-    {
-      float lo, hi;
-      f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
-      l_run += lo + hi;
-    }
     if constexpr (kF8) {
       tmem_st_x32(tS, pk);
     } else {
@@ -407,6 +411,16 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     tmem_st_wait();
     tc_fence_before_sync();
     mbar_arrive(bar_p_ready);
+    // The row sum of the fp32 weights (kept in sr) is taken after P is handed
+    // over: it runs while the tensor core works on this tile's P.V.
+#pragma unroll
+    for (int cc = 0; cc < 64; ++cc)
+      acc[cc % 4] = f2_add(acc[cc % 4], f2_pack(__uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1])));
+    {
+      float lo, hi;
+      f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
+      l_run += lo + hi;
+    }
   }
   if constexpr (!kKV) {
     if (ok) ok = warp_wait(bar_o_final, 0, wd);
@@ -603,33 +617,41 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   // S_g = Q_g K^T : A = Q tile (K-major), B = K tile (K-major); each
   // instruction reduces 32 bytes of d (16 bf16 or 32 E4M3 values), stepping
   // through the 128-byte swizzle atoms of a row.
+  // The shared-memory descriptors of one launch differ only in their start
+  // address (the low word; the high word holds the stride, version and
+  // swizzle): keep the low words of the three bases, add each operand's
+  // offset to them and attach the common high word, a few integer operations
+  // per MMA for the single issuing thread.
+  const uint64_t kk_hi = sdesc_sw128(0, 16, 1024) & 0xFFFFFFFF00000000ull;
+  const uint32_t q_lo = static_cast<uint32_t>(sdesc_sw128(sQ, 16, 1024));
+  const uint32_t r_lo = static_cast<uint32_t>(sdesc_sw128(sRing, 16, 1024));
+  const uint32_t v_lo = static_cast<uint32_t>(sdesc_sw128(sRing, C::kAtomBytes, 1024));
+  auto mk = [&](uint32_t lo) { return kk_hi | lo; };
   auto issue_qk = [&](int g, int slot) {
-    const uint32_t a0 = sQ + g * C::kTileBytes;
-    const uint32_t b0 = sRing + slot * C::kTileBytes;
+    const uint32_t a0 = q_lo + static_cast<uint32_t>((g * C::kTileBytes) >> 4);
+    const uint32_t b0 = r_lo + static_cast<uint32_t>((slot * C::kTileBytes) >> 4);
 #pragma unroll
     for (int kk = 0; kk < D / C::kMmaK; ++kk) {
-      const uint32_t off = (kk >> 2) * C::kAtomBytes + (kk & 3) * 32;
+      const uint32_t off = ((kk >> 2) * C::kAtomBytes + (kk & 3) * 32) >> 4;
       if constexpr (kF8)
-        mma_ss_f8(tmem + C::col_s(g), sdesc_sw128(a0 + off, 16, 1024),
-                  sdesc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        mma_ss_f8(tmem + C::col_s(g), mk(a0 + off), mk(b0 + off), idesc_qk, kk > 0 ? 1u : 0u);
       else
-        mma_ss(tmem + C::col_s(g), sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
-               idesc_qk, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + C::col_s(g), mk(a0 + off), mk(b0 + off), idesc_qk, kk > 0 ? 1u : 0u);
     }
   };
   // O_g += P_g V : A = P in tensor memory (8 columns per instruction: 16 bf16
   // or 32 E4M3 keys), B = V tile (MN-major, rows of 128 bytes, one per key).
   auto issue_pv = [&](int g, int slot, bool accumulate) {
-    const uint32_t b0 = sRing + slot * C::kTileBytes;
+    const uint32_t b0 = v_lo + static_cast<uint32_t>((slot * C::kTileBytes) >> 4);
 #pragma unroll
     for (int kk = 0; kk < kTileRows / C::kMmaK; ++kk) {
       if constexpr (kF8)
         mma_ts_f8(tmem + C::col_o(g), tmem + C::col_s(g) + kk * 8,
-                  sdesc_sw128(b0 + kk * C::kMmaK * 128, C::kAtomBytes, 1024), idesc_pv,
+                  mk(b0 + static_cast<uint32_t>((kk * C::kMmaK * 128) >> 4)), idesc_pv,
                   (accumulate || kk > 0) ? 1u : 0u);
       else
         mma_ts(tmem + C::col_o(g), tmem + C::col_s(g) + kk * 8,
-               sdesc_sw128(b0 + kk * 2048, C::kAtomBytes, 1024), idesc_pv,
+               mk(b0 + static_cast<uint32_t>((kk * 2048) >> 4)), idesc_pv,
                (accumulate || kk > 0) ? 1u : 0u);
     }
   };
@@ -647,7 +669,7 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
     const int u = j + 1;  // V_j and K_{j+1}
     if (!(ok = wait_one(full_bar(u), par_of(u), wd))) break;
     if (j < na) {
-      if (!(ok = wait_one(bar_p_ready0, j & 1, wd))) break;
+      if (!(ok = wait_spin(bar_p_ready0, j & 1, wd))) break;
       tc_fence_after_sync();
       issue_pv(0, v_slot(u), j > 0);
       if (j + 1 < na) {
@@ -657,7 +679,7 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
         mma_commit(bar_o_final0);
       }
     }
-    if (!(ok = wait_one(bar_p_ready0 + 8u, j & 1, wd))) break;
+    if (!(ok = wait_spin(bar_p_ready0 + 8u, j & 1, wd))) break;
     tc_fence_after_sync();
     issue_pv(1, v_slot(u), j > 0);
     if (j + 1 < nb) {
@@ -1011,6 +1033,8 @@ bool current_context_id(unsigned long long* id) {
 
 namespace {
 
+unsigned int* device_error_word();
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -1045,6 +1069,25 @@ bool encode_qkv_map(CUtensorMap* m, const void* ptr, int BH, int N, int d, int e
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+bool encode_bf16_tiled_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                          uint32_t box0, uint32_t box1) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+unsigned int* library_error_word() { return device_error_word(); }
+
+namespace {
 
 // Device address of g_device_error in the current context.
 unsigned int* device_error_word() {

@@ -1,6 +1,7 @@
 // internal.h - host-side entry points shared by the translation units of
 // libattn_b200.so (not part of the public C ABI; see include/attn.h).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -85,6 +86,13 @@ void* noalloc_scratch_ptr();
 // now on (fused_fwd.cu); default 2000 ms.
 void set_wait_limit_ms(int ms);
 int wait_limit_ms();
+
+// Tensor map of a [d2][d1][d0] bf16 array (d0 innermost), box {box0, box1, 1},
+// 128-byte swizzle, zero fill out of bounds (fused_fwd.cu).
+bool encode_bf16_tiled_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                          uint32_t box0, uint32_t box1);
+// Address of the device error word in the current context, or null.
+unsigned int* library_error_word();
 
 // Device error word of the current device (fused_fwd.cu).
 int read_and_clear_device_error(cudaStream_t stream);

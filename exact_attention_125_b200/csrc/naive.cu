@@ -8,8 +8,9 @@
 //   3. values:  O = P V (fp32 accumulate, bf16 out)                       -> HBM
 // The N x N matrices S and P each cross the HBM boundary twice. This path is
 // a measuring stick for that traffic, not a product path: its two matrix
-// products use warp-level mma.sync tensor-core instructions so that it is
-// bound by memory, as the pages say it is, rather than by scalar arithmetic.
+// products run on the tensor cores (tcgen05 with TMA-fed tiles when N % 8 ==
+// 0, warp-level mma.sync otherwise) so that it is bound by memory, as the
+// pages say it is, rather than by arithmetic.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -19,6 +20,9 @@
 #include "../../include/attn.h"
 #include "ctx_cache.h"
 #include "internal.h"
+#include "sm100.cuh"
+#include "tmem_io.cuh"
+#include "watchdog.cuh"
 
 namespace attn {
 namespace {
@@ -348,6 +352,373 @@ __global__ void __launch_bounds__(256) naive_values_kernel(const uint16_t* __res
     }
 }
 
+// ------------------------------------------- tcgen05 kernels (N % 8 == 0)
+// The same two matrix products on the 5th-generation tensor cores, with TMA
+// moving every tile: S row blocks stream out of shared memory through TMA
+// stores, P and V tiles stream in through TMA loads, so the products keep up
+// with HBM and the path's time is the traffic it is there to show. (S and P
+// are [B*H, N, N] bf16 arrays; a TMA row stride must be a multiple of 16
+// bytes, hence N % 8 == 0; other N take the kernels above.)
+//
+// Roles (192 threads): warp 0 TMA producer, warp 1 tensor-memory allocator
+// and MMA issuer, warps 2-5 epilogue (thread = tile row; warp w reaches
+// tensor-memory lanes 32 (w % 4) .. + 31).
+constexpr int kTcThreads = 192;
+
+struct TcBars {
+  // byte offsets of the mbarriers from the barrier area
+  __host__ __device__ static constexpr uint32_t full(int s) { return 8u * s; }  // s < 4
+  __host__ __device__ static constexpr uint32_t empty(int s) { return 8u * (4 + s); }
+  __host__ __device__ static constexpr uint32_t acc_full(int b) { return 8u * (8 + b); }  // b < 2
+  __host__ __device__ static constexpr uint32_t acc_empty(int b) { return 8u * (10 + b); }
+  static constexpr uint32_t kQFull = 8u * 12;
+  static constexpr uint32_t kMmaDone = 8u * 13;
+  static constexpr int kCount = 14;
+};
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// S = scale * Q K^T for 128 query rows of one head (all N keys), written to
+// HBM as bf16 with causally masked entries -inf. The tensor core fills one of
+// two S buffers in tensor memory while the epilogue drains the other into a
+// swizzled staging tile that two TMA stores (64 columns each) copy out.
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    naive_scores_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                           const __grid_constant__ CUtensorMap ts, int N, int nqb, float scale,
+                           int causal, unsigned int* err, uint64_t wait_limit_ns) {
+  constexpr int kTile = kT * D * 2;            // Q or K tile bytes
+  constexpr int kAtom = kT * 128;              // 128 rows x 128 bytes
+  constexpr int kStages = 3;
+  constexpr int kStage = kT * kT * 2;          // staging tile, 32 KiB (two atoms)
+  constexpr uint32_t kRingOff = kTile, kStageOff = kRingOff + kStages * kTile;
+  constexpr uint32_t kBarOff = kStageOff + 2 * kStage;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - smem_addr(smem_raw));
+  const uint32_t bars = base + kBarOff;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * TcBars::kCount);
+  volatile uint32_t* abort_flag = misc + 1;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.x / nqb, r0 = (blockIdx.x % nqb) * kT;
+  const int T = (N + kT - 1) / kT;
+  // key tiles with at least one allowed key for some row of the block
+  const int n_mma = causal ? min(T, r0 / kT + 1) : T;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(bars + TcBars::full(i), 1);
+      mbar_init(bars + TcBars::empty(i), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bars + TcBars::acc_full(b), 1);
+      mbar_init(bars + TcBars::acc_empty(b), 128);
+    }
+    mbar_init(bars + TcBars::kQFull, 1);
+    mbar_init(bars + TcBars::kMmaDone, 1);
+    *abort_flag = 0u;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(misc), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc);
+  const Watchdog wd{abort_flag, err, wait_limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();
+      mbar_arrive_expect_tx(bars + TcBars::kQFull, kTile);
+      for (int a = 0; a < D / 64; ++a)
+        tma_load_3d_hint(base + a * kAtom, &tq, bars + TcBars::kQFull, a * 64, r0, bh, pol);
+      int j = 0;
+      for (; j < n_mma; ++j) {
+        const int s = j % kStages;
+        if (!wait_one(bars + TcBars::empty(s), ((j / kStages) & 1) ^ 1u, wd)) break;
+        mbar_arrive_expect_tx(bars + TcBars::full(s), kTile);
+        for (int a = 0; a < D / 64; ++a)
+          tma_load_3d_hint(base + kRingOff + s * kTile + a * kAtom, &tk, bars + TcBars::full(s), a * 64,
+                           j * kT, bh, pol);
+      }
+      drain_wait(bars + TcBars::kQFull, 0, wd);
+      for (int w = (j > kStages ? j - kStages : 0); w < j; ++w)
+        drain_wait(bars + TcBars::full(w % kStages), (w / kStages) & 1, wd);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      bool ok = wait_one(bars + TcBars::kQFull, 0, wd);
+      for (int j = 0; ok && j < n_mma; ++j) {
+        const int s = j % kStages, b = j & 1;
+        if (!(ok = wait_one(bars + TcBars::full(s), (j / kStages) & 1, wd))) break;
+        if (!(ok = wait_one(bars + TcBars::acc_empty(b), ((j >> 1) & 1) ^ 1u, wd))) break;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+          mma_ss(tmem + 128u * b, sdesc_sw128(base + off, 16, 1024),
+                 sdesc_sw128(base + kRingOff + s * kTile + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bars + TcBars::acc_full(b));
+        mma_commit(bars + TcBars::empty(s));
+      }
+      mma_commit(bars + TcBars::kMmaDone);
+      drain_wait(bars + TcBars::kMmaDone, 0, wd);
+    }
+  } else {
+    // epilogue: thread = row r of the block
+    const int r = 32 * (warp % 4) + lane;
+    const int row = r0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp % 4)) << 16;
+    const bool leader = threadIdx.x == 64;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int b = j & 1;
+      const uint32_t stage = base + kStageOff + b * kStage;
+      // the store that last read this staging tile (two tiles ago) has finished reading
+      if (leader) bulk_wait_read<1>();
+      named_barrier_sync(1, 128);
+      const int col0 = j * kT;
+      if (j < n_mma) {
+        if (ok) ok = warp_wait(bars + TcBars::acc_full(b), (j >> 1) & 1, wd);
+        tc_fence_after_sync();
+        const int lim = causal ? row - col0 : kT;  // columns cc > lim are masked
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t v[32];
+          if (ok) tmem_ld_x32_wait(tmem + lane_base + 128u * b + ch * 32, v);
+          uint32_t w[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int c = ch * 32 + 2 * u;
+            const float s0 = c > lim ? -INFINITY : __uint_as_float(v[2 * u]) * scale;
+            const float s1 = c + 1 > lim ? -INFINITY : __uint_as_float(v[2 * u + 1]) * scale;
+            w[u] = bf16x2_bits(s0, s1);
+          }
+          // 16-byte chunk q of this row's 64-column atom goes to chunk q ^ (r & 7)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (ch % 2) * 4 + q;
+            uint8_t* dst = smem + (stage - base) + (ch / 2) * kAtom + r * 128 + ((chunk ^ (r & 7)) * 16);
+            *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(bars + TcBars::acc_empty(b));
+      } else {
+        // every key of the tile is after every row of the block: all -inf
+        const uint4 ninf = make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          *reinterpret_cast<uint4*>(smem + (stage - base) + (q / 8) * kAtom + r * 128 + (q % 8) * 16) = ninf;
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 128);
+      if (leader) {
+        tma_store_3d(&ts, stage, col0, r0, bh);
+        if (col0 + 64 < N) tma_store_3d(&ts, stage + kAtom, col0 + 64, r0, bh);
+        bulk_commit();
+      }
+    }
+    if (leader) bulk_wait_all();
+  }
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// O = P V for 128 query rows of one head: P and V tiles of 128 keys stream
+// through a ring (every P tile is read, as the unfused algorithm reads all of
+// P; tiles wholly above the causal diagonal are all zero and skip the MMA).
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    naive_values_tc_kernel(const __grid_constant__ CUtensorMap tp, const __grid_constant__ CUtensorMap tv,
+                           uint16_t* __restrict__ O, int N, int nqb, int causal, unsigned int* err,
+                           uint64_t wait_limit_ns) {
+  constexpr int kPTile = kT * kT * 2;          // 32 KiB
+  constexpr int kVTile = kT * D * 2;
+  constexpr int kAtom = kT * 128;
+  constexpr int kUnit = kPTile + kVTile;
+  constexpr int kStages = 3;
+  constexpr uint32_t kBarOff = kStages * kUnit;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - smem_addr(smem_raw));
+  const uint32_t bars = base + kBarOff;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * TcBars::kCount);
+  volatile uint32_t* abort_flag = misc + 1;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.x / nqb, r0 = (blockIdx.x % nqb) * kT;
+  const int T = (N + kT - 1) / kT;
+  const int n_mma = causal ? min(T, r0 / kT + 1) : T;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(bars + TcBars::full(i), 1);
+      mbar_init(bars + TcBars::empty(i), 1);
+    }
+    mbar_init(bars + TcBars::acc_full(0), 1);
+    mbar_init(bars + TcBars::kMmaDone, 1);
+    *abort_flag = 0u;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(misc), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc);
+  const Watchdog wd{abort_flag, err, wait_limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_p = l2_policy_evict_first();
+      const uint64_t pol_v = l2_policy_evict_last();
+      int j = 0;
+      for (; j < T; ++j) {
+        const int s = j % kStages;
+        if (!wait_one(bars + TcBars::empty(s), ((j / kStages) & 1) ^ 1u, wd)) break;
+        const uint32_t unit = base + s * kUnit;
+        mbar_arrive_expect_tx(bars + TcBars::full(s), kUnit);
+        for (int a = 0; a < 2; ++a)
+          tma_load_3d_hint(unit + a * kAtom, &tp, bars + TcBars::full(s), j * kT + a * 64, r0, bh, pol_p);
+        for (int a = 0; a < D / 64; ++a)
+          tma_load_3d_hint(unit + kPTile + a * kAtom, &tv, bars + TcBars::full(s), a * 64, j * kT, bh,
+                           pol_v);
+      }
+      for (int w = (j > kStages ? j - kStages : 0); w < j; ++w)
+        drain_wait(bars + TcBars::full(w % kStages), (w / kStages) & 1, wd);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+      bool ok = true;
+      for (int j = 0; ok && j < T; ++j) {
+        const int s = j % kStages;
+        if (!(ok = wait_one(bars + TcBars::full(s), (j / kStages) & 1, wd))) break;
+        if (j < n_mma) {
+          tc_fence_after_sync();
+          const uint32_t unit = base + s * kUnit;
+#pragma unroll
+          for (int kk = 0; kk < kT / 16; ++kk) {
+            // A = P tile (K-major: 128 rows, keys in two 128-byte atoms), B =
+            // V tile (MN-major: one 128-byte row of d per key)
+            const uint32_t a_off = (kk >> 2) * kAtom + (kk & 3) * 32;
+            mma_ss(tmem, sdesc_sw128(unit + a_off, 16, 1024),
+                   sdesc_sw128(unit + kPTile + kk * 2048, kAtom, 1024), idesc,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(bars + TcBars::empty(s));
+      }
+      mma_commit(bars + TcBars::acc_full(0));
+      mma_commit(bars + TcBars::kMmaDone);
+      drain_wait(bars + TcBars::kMmaDone, 0, wd);
+    }
+  } else {
+    const int r = 32 * (warp % 4) + lane;
+    const int row = r0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp % 4)) << 16;
+    if (warp_wait(bars + TcBars::acc_full(0), 0, wd)) {
+      tc_fence_after_sync();
+      uint16_t* orow = O + (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld_x32_wait(tmem + lane_base + ch * 32, v);
+        if (row < N) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(orow + ch * 32 + q * 8) = make_uint4(
+                bf16x2_bits(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                bf16x2_bits(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                bf16x2_bits(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                bf16x2_bits(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+template <int D>
+int launch_naive_tc(const AttnArgs& a, uint16_t* S, uint16_t* P, float* lse, cudaStream_t stream,
+                    int softmax_ept, int softmax_threads) {
+  const int N = a.N, BH = a.B * a.H;
+  const int nqb = (N + kT - 1) / kT;
+  CUtensorMap mq, mk, ms, mp, mv;
+  if (!encode_bf16_tiled_3d(&mq, a.q, D, N, BH, 64, kT) || !encode_bf16_tiled_3d(&mk, a.k, D, N, BH, 64, kT) ||
+      !encode_bf16_tiled_3d(&ms, S, N, N, BH, 64, kT) || !encode_bf16_tiled_3d(&mp, P, N, N, BH, 64, kT) ||
+      !encode_bf16_tiled_3d(&mv, a.v, D, N, BH, 64, kT))
+    return ATTN_ERR_CUDA;
+  unsigned int* err = library_error_word();
+  if (!err) return ATTN_ERR_CUDA;
+  const uint64_t limit = static_cast<uint64_t>(wait_limit_ms()) * 1000000ull;
+  const long long grid = static_cast<long long>(nqb) * BH;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+  static CtxCache<int> prep;
+  int st = ATTN_ERR_CUDA;
+  constexpr int kScoresSmem = kT * D * 2 * 4 + 2 * kT * kT * 2 + 8 * TcBars::kCount + 16 + 1024;
+  constexpr int kValuesSmem = 3 * (kT * kT * 2 + kT * D * 2) + 8 * TcBars::kCount + 16 + 1024;
+  static_assert(kScoresSmem <= 227 * 1024 && kValuesSmem <= 227 * 1024, "shared memory");
+  if (!prep.get(&st, [](int* out) {
+        *out = (cudaFuncSetAttribute(naive_scores_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kScoresSmem) == cudaSuccess &&
+                cudaFuncSetAttribute(naive_values_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kValuesSmem) == cudaSuccess)
+                   ? ATTN_OK
+                   : ATTN_ERR_CUDA;
+        return *out == ATTN_OK;
+      }))
+    return ATTN_ERR_CUDA;
+  naive_scores_tc_kernel<D><<<static_cast<unsigned>(grid), kTcThreads, kScoresSmem, stream>>>(
+      mq, mk, ms, N, nqb, a.scale, a.causal, err, limit);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  const unsigned rows = static_cast<unsigned>(static_cast<size_t>(BH) * N);
+  switch (softmax_ept) {
+    case 8: naive_softmax_kernel<8><<<rows, softmax_threads, 0, stream>>>(S, P, lse, N); break;
+    case 16: naive_softmax_kernel<16><<<rows, softmax_threads, 0, stream>>>(S, P, lse, N); break;
+    case 32: naive_softmax_kernel<32><<<rows, softmax_threads, 0, stream>>>(S, P, lse, N); break;
+    default: naive_softmax_kernel<64><<<rows, softmax_threads, 0, stream>>>(S, P, lse, N); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  naive_values_tc_kernel<D><<<static_cast<unsigned>(grid), kTcThreads, kValuesSmem, stream>>>(
+      mp, mv, static_cast<uint16_t*>(a.o), N, nqb, a.causal, err, limit);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
 template <int D>
 int launch_naive_d(const AttnArgs& a, void* workspace, cudaStream_t stream) {
   const int N = a.N, BH = a.B * a.H;
@@ -358,6 +729,12 @@ int launch_naive_d(const AttnArgs& a, void* workspace, cudaStream_t stream) {
   const auto* v = static_cast<const uint16_t*>(a.v);
   auto* o = static_cast<uint16_t*>(a.o);
   const int tiles = (N + kT - 1) / kT;
+  // softmax launch shape: EPT elements per thread, T threads per row
+  int ept = 8;
+  while (ept < 64 && (N + ept - 1) / ept > 256) ept *= 2;
+  const int T = ((N + ept - 1) / ept + 31) / 32 * 32;
+  if (T > 512) return ATTN_ERR_SHAPE;
+  if (N % 8 == 0) return launch_naive_tc<D>(a, S, P, a.lse, stream, ept, T);
   if (BH > 65535) return ATTN_ERR_SHAPE;
 
   const int smem_scores = 2 * kT * (D + 8) * 2;
@@ -368,11 +745,6 @@ int launch_naive_d(const AttnArgs& a, void* workspace, cudaStream_t stream) {
                                                                               a.causal);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
 
-  // softmax launch shape: EPT elements per thread, T threads per row
-  int ept = 8;
-  while (ept < 64 && (N + ept - 1) / ept > 256) ept *= 2;
-  int T = ((N + ept - 1) / ept + 31) / 32 * 32;
-  if (T > 512) return ATTN_ERR_SHAPE;
   const unsigned rows = static_cast<unsigned>(static_cast<size_t>(BH) * N);
   switch (ept) {
     case 8: naive_softmax_kernel<8><<<rows, T, 0, stream>>>(S, P, a.lse, N); break;

@@ -57,6 +57,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same condition (try_wait may suspend the thread for
+// a while when the phase is not complete; test_wait returns at once).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // --------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -223,6 +237,11 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // complement) into the exponent field and drops everything else. Inputs are
 // clamped at -125 so the result stays a positive number (2^-125 ~ 2e-38 stands
 // in for 0 when x = -inf); relative error <= kExp2PolyMaxRelErr + fp32 rounding.
+// So a masked logit (-inf) on these columns gives a weight of 2^-125, not 0.
+// The callers rely on what follows: a row's sum l >= 1 once it has seen an
+// allowed key (2^-125 is then lost in fp32 rounding of l and of O), and a row
+// that has seen none (m = -inf, only possible in a split of the kv path) has
+// its l reset to 0 before the epilogue, which writes O = 0 and lse = -inf.
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -125.0f);
   const float t = __fadd_rn(x, 12582912.0f);

@@ -28,6 +28,24 @@ __device__ __forceinline__ bool timed_out(uint64_t t0, const Watchdog& w) {
   return true;
 }
 
+// Wait by the MMA-issuing thread for a softmax hand-off: spins on test_wait
+// (which never suspends the thread) and checks the abort flag and the time
+// limit every 64 polls. try_wait may suspend a thread for a while after the
+// phase completes; on the MMA thread that latency sits on every step's
+// critical path (measured: the spinning issuer wakes ~100-150 cycles sooner
+// after a long wait).
+__device__ __forceinline__ bool wait_spin(uint32_t bar, uint32_t parity, const Watchdog& w) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 63) == 63) {
+      if (t0 == 0) t0 = global_timer_ns();
+      if (*w.abort) return false;
+      if (timed_out(t0, w)) return false;
+    }
+  }
+}
+
 // Wait by a single thread (TMA producer, MMA issuer).
 __device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, const Watchdog& w) {
   if (mbar_try_wait(bar, parity)) return true;

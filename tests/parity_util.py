@@ -52,7 +52,7 @@ def max_abs_logit(q, k, scale, causal, rows):
     for bh in np.unique(rows[:, 0]):
         sel = np.nonzero(rows[:, 0] == bh)[0]
         i = torch.as_tensor(rows[sel, 1])
-        s = (qf[bh, i] @ kf[bh].T).abs() * scale
+        s = (qf[bh, i] @ kf[bh].T).abs() * abs(scale)
         if causal:
             s = s.masked_fill(torch.arange(N)[None, :] > i[:, None], 0.0)
         out[sel] = s.max(dim=1).values.numpy()

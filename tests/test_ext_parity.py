@@ -12,7 +12,7 @@ import torch
 
 import exact_attention_125_b200 as ea
 import oracle
-from exact_attention_125_b200.inputs import gather_rows, make_q_kv
+from exact_attention_125_b200.inputs import gather_rows, make_q_kv, sample_rows
 from parity_util import assert_within, compare, scale_of
 
 pytestmark = pytest.mark.gpu
@@ -91,3 +91,31 @@ def test_ext_without_options_matches_attn_fwd_kv_bit_for_bit():
     o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=True, num_splits=3)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("B,H,N,wl,alibi", [
+    # the benchmark's two shapes with fewer heads: a 4096-key sliding window
+    # over a 32768-token causal prefill, and the distance bias at 8192 (the
+    # slopes of the benchmark's 32 heads, first eight)
+    (1, 4, 32768, 4095, False),
+    (1, 8, 8192, -1, True),
+])
+def test_benchmark_shapes_sampled_rows(B, H, N, wl, alibi):
+    d = 128
+    q, k, v = make_q_kv(B, H, N, N, d, seed=N + wl + int(alibi))
+    slopes = [2.0 ** (-8.0 * (h + 1) / 32) for h in range(H)] if alibi else None
+    qg, kg, vg = (t.to("cuda") for t in (q, k, v))
+    sl = torch.tensor(slopes, dtype=torch.float32, device="cuda") if slopes else None
+    o = torch.full((B, H, N, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device="cuda")
+    # automatic split count, as the benchmark launches it
+    ea.attn_fwd_ext(qg, kg, vg, o, lse, scale=scale_of(d), causal=True, window_left=wl,
+                    alibi_slopes=sl, num_splits=0)
+    torch.cuda.synchronize()
+    assert ea.last_device_error() == 0
+    rows = sample_rows(N + 17, B * H, N, 64)
+    sl64 = [float(np.float32(x)) for x in slopes] if slopes else None
+    o_ref, lse_ref = oracle.attention_ext(q, k, v, scale_of(d), True, wl, -1, sl64, rows=rows)
+    e = compare(gather_rows(o.cpu(), rows), gather_rows(lse.cpu().unsqueeze(-1), rows).squeeze(-1),
+                o_ref, lse_ref)
+    assert_within(e, f"bench shape {(B, H, N, wl, alibi)}")
