@@ -80,9 +80,15 @@ constexpr int kMmaWarp = 9;     // warps 10 and 11 only give their registers awa
 // host refuses to launch otherwise), and the split after setmaxnreg. The
 // split uses exactly the launch total.
 constexpr int kRegsAtLaunch = 168;
-constexpr int kRegsSoftmax = 224;
-constexpr int kRegsOther = 56;
-static_assert(128 * (2 * kRegsSoftmax + kRegsOther) == kThreads * kRegsAtLaunch,
+// kv path: 224 for each softmax warpgroup, 56 for the producer/MMA one; the
+// persistent square path gives the producer and MMA warps 88 for their work
+// loop (its softmax fits in 208).
+template <bool kKV>
+constexpr int kRegsSoftmax = kKV ? 224 : 216;
+template <bool kKV>
+constexpr int kRegsOther = kKV ? 56 : 72;
+static_assert(128 * (2 * kRegsSoftmax<true> + kRegsOther<true>) == kThreads * kRegsAtLaunch &&
+                  128 * (2 * kRegsSoftmax<false> + kRegsOther<false>) == kThreads * kRegsAtLaunch,
               "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 256 while m lags
@@ -121,10 +127,17 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_final[2], mma_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 6 + 1;
+  // q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_final[2],
+  // mma_done, q_empty (square path: the Q tiles may be overwritten),
+  // stage_free (square path: the O staging tile may be overwritten)
+  static constexpr int kNumBars = 1 + 2 * kStages + 6 + 3;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;  // tmem base, abort flag
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;   // + alignment slack
+  // square path: one bf16 O tile (128 rows, 128-byte swizzle atoms of 64
+  // columns) staged for its TMA store, after the barriers, 1024-aligned
+  static constexpr int kStageOff = (kMiscOff + 16 + 1023) / 1024 * 1024;
+  static constexpr int kStageBytes = kTileRows * D * 2;
+  static constexpr int kSmemBytes = kStageOff + kStageBytes + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "square path exceeds the shared memory of a CTA");
   // kv path: (m, l) of every softmax thread, swapped between the two
   // warpgroups when they took alternate KV tiles of one query tile
   static constexpr int kXchOff = kMiscOff + 16;
@@ -230,10 +243,16 @@ __device__ __forceinline__ void store_row_chunk(const FwdParams& p, bool partial
 
 // ctl: shared address of the control barriers s_full[2], p_ready[2],
 // o_final[2] (consecutive).
+// s_phase0: steps this warpgroup has taken before (the square path's work
+// units follow one another on the same barriers); o_phase: parity of this
+// unit's o_final phase. Returns false once a wait has given up.
 template <int D, bool kKV, bool kF8 = false>
-__device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, uint32_t ctl,
+__device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, uint32_t ctl,
                                              int bh, int q0, int n_kv, int g,
-                                             const Watchdog& wd, int kv_lo) {
+                                             const Watchdog& wd, int kv_lo, uint32_t s_phase0 = 0,
+                                             uint32_t o_phase = 0,
+                                             const CUtensorMap* tmap_o = nullptr,
+                                             uint32_t stage = 0, uint32_t stage_use = 0) {
   using C = Cfg<D, kF8>;
   const int warp = threadIdx.x / 32;
   const int tid = threadIdx.x % 128;
@@ -279,7 +298,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
   float l_run = 0.0f;
   bool ok = true;
   for (int j = 0; j < n_kv; ++j) {
-    if (!(ok = warp_wait(bar_s_full, j & 1, wd))) break;
+    if (!(ok = warp_wait(bar_s_full, (s_phase0 + j) & 1, wd))) break;
     tc_fence_after_sync();
     uint32_t sr[128];
     tmem_ld_x128_wait(tS, sr);
@@ -391,8 +410,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
         p0 = ex2_approx(x0);
         p1 = ex2_approx(x1);
       }
-      sr[2 * cc] = __float_as_uint(p0);
-      sr[2 * cc + 1] = __float_as_uint(p1);
+      acc[cc % 4] = f2_add(acc[cc % 4], f2_pack(p0, p1));
       if constexpr (kF8) {
         const uint32_t h = pack_e4m3x2(p0, p1);
         if (cc % 2 == 0)
@@ -411,11 +429,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     tmem_st_wait();
     tc_fence_before_sync();
     mbar_arrive(bar_p_ready);
-    // The row sum of the fp32 weights (kept in sr) is taken after P is handed
-    // over: it runs while the tensor core works on this tile's P.V.
-#pragma unroll
-    for (int cc = 0; cc < 64; ++cc)
-      acc[cc % 4] = f2_add(acc[cc % 4], f2_pack(__uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1])));
     {
       float lo, hi;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), lo, hi);
@@ -423,15 +436,26 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     }
   }
   if constexpr (!kKV) {
-    if (ok) ok = warp_wait(bar_o_final, 0, wd);
-    if (!ok) return;
+    if (ok) ok = warp_wait(bar_o_final, o_phase, wd);
+    if (!ok) return false;
     tc_fence_after_sync();
 
-    // Epilogue: O / l -> bf16 (times V's scale on the FP8 path), lse in natural log.
+    // Epilogue: O / l -> bf16 (times V's scale on the FP8 path), lse in natural
+    // log. The O tile goes through a shared staging tile (128-byte swizzle,
+    // so the row-per-thread writes are free of bank conflicts) and leaves in
+    // TMA stores of whole lines; writing rows straight from registers cost
+    // ~16 partial-line stores per thread, thousands of cycles per tile. Both
+    // query tiles and all work units of the CTA share the staging tile, in
+    // turn: use u waits until the store of use u - 1 has read it.
     const float inv_l = kF8 ? p.v_descale / l_run : 1.0f / l_run;
     const bool valid = row < p.N;
-    uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
-                                           (static_cast<size_t>(bh) * p.N + row) * D);
+    const uint32_t bar_stage_free = ctl + 64u;
+    if (stage_use > 0 && !warp_wait(bar_stage_free, (stage_use - 1) & 1, wd)) return false;
+    uint8_t* stage_ptr = nullptr;
+    {
+      extern __shared__ uint8_t smem_raw[];
+      stage_ptr = smem_raw + (stage - smem_u32(smem_raw));
+    }
 #pragma unroll
     for (int ch = 0; ch < D / 32; ++ch) {
       uint32_t orr[32];
@@ -440,11 +464,25 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         w[u] = pack_bf16x2(__uint_as_float(orr[2 * u]) * inv_l, __uint_as_float(orr[2 * u + 1]) * inv_l);
-      if (valid) {
+      // 16-byte chunk q of the row's 64-column atom goes to chunk q ^ (row & 7)
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          orow[ch * 4 + u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      for (int q = 0; q < 4; ++q) {
+        const int chunk = (ch % 2) * 4 + q;
+        *reinterpret_cast<uint4*>(stage_ptr + (ch / 2) * (kTileRows * 128) + tid * 128 +
+                                  ((chunk ^ (tid & 7)) * 16)) =
+            make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
       }
+    }
+    fence_proxy_async_smem();
+    named_barrier_sync(2 + g, 128);
+    if (tid == 0) {
+      // rows past N are clipped by the store
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a)
+        tma_store_3d(tmap_o, stage + a * (kTileRows * 128), a * 64, row_start, bh);
+      bulk_commit();
+      bulk_wait_read<0>();
+      mbar_arrive(bar_stage_free);
     }
     if (valid) {
       const float m_fin = (m_run == -INFINITY) ? 0.0f : m_run;
@@ -465,7 +503,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
     const uint32_t bar_o_final0 = ctl + 8u * 4;
     if (!alt) {
       if (ok && n_kv > 0) ok = warp_wait(bar_o_final, 0, wd);
-      if (!ok) return;
+      if (!ok) return false;
       tc_fence_after_sync();
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
 #pragma unroll
@@ -499,7 +537,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
       xch[2 * (128 * g + tid)] = m_run;
       xch[2 * (128 * g + tid) + 1] = l_run;
       named_barrier_sync(1, 256);
-      if (*wd.abort) return;
+      if (*wd.abort) return false;
       tc_fence_after_sync();
       const float m_o = xch[2 * (128 * (1 - g) + tid)];
       const float l_o = xch[2 * (128 * (1 - g) + tid) + 1];
@@ -537,64 +575,123 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t tmem, 
         lse_dst[row_index] = L > 0.0f ? (m + __log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
   }
+  return ok;
 }
 
+// Square path work units. The query blocks (256 rows) of a head are paired
+// heaviest with lightest, (nqb - 1 - i, i): causally every pair then costs the
+// same number of KV steps, so dealing the pairs to the CTAs in turn (CTA c
+// takes pairs c, c + gridDim.x, ...) balances the SMs without a global work
+// counter, and pairs are head-major so the CTAs running at the same time share
+// K/V in L2. Unit k of the CTA is half k % 2 of its pair k / 2 (the heavy
+// block first); with nqb odd the middle block of a head forms a pair alone.
+// Every role of the CTA walks the same sequence.
+struct SquareUnit {
+  int bh, q0, na, nb;
+};
+
+// k: the CTA's unit index, advanced past a skipped (absent) second half.
+__device__ __forceinline__ bool square_unit(const FwdParams& p, int& k, SquareUnit& u) {
+  const int npairs = (p.nqb + 1) / 2;
+  while (true) {
+    const int pair = static_cast<int>(blockIdx.x) + (k / 2) * static_cast<int>(gridDim.x);
+    if (pair >= npairs * p.BH) return false;
+    const int i = pair % npairs;
+    const int qblk = (k % 2 == 0) ? p.nqb - 1 - i : i;
+    if (k % 2 == 1 && qblk == p.nqb - 1 - i) {  // the middle block of an odd nqb
+      ++k;
+      continue;
+    }
+    u.bh = pair / npairs;
+    u.q0 = qblk * kBlockRows;
+    u.na = p.causal ? min(p.T, u.q0 / kTileRows + 1) : p.T;
+    u.nb = p.causal ? min(p.T, u.q0 / kTileRows + 2) : p.T;
+    return true;
+  }
+}
+
+// Square path producer: for each of the CTA's work units, the K/V units of
+// its KV tiles (unit 0 = K_0, unit u >= 1 = (V_{u-1}, K_u), the last V only)
+// into the ring, which runs on across work units, and the unit's two Q tiles
+// once the previous unit's last Q K^T has completed (q_empty). K_0 of the next
+// unit is requested before that wait, so both arrive while the current unit's
+// last step is still running.
 template <int D, bool kF8 = false>
 __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUtensorMap* tk,
                                               const CUtensorMap* tv, uint32_t base, uint32_t bars,
-                                              int bh, int q0, int n_kv_b, const Watchdog& wd) {
+                                              const FwdParams& p, const Watchdog& wd) {
   using C = Cfg<D, kF8>;
   const uint32_t sQ = base + C::kQOff;
   const uint32_t sRing = base + C::kRingOff;
   const uint32_t bar_q = bars;
+  const uint32_t bar_q_empty = bars + 8u * (1 + 2 * C::kStages + 7);
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-
-  mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
+  int ug = 0;    // ring position, across work units
+  int done = 0;  // work units of this CTA so far
+  bool ok = true;
+  SquareUnit cur;
+  for (int k = 0; ok && square_unit(p, k, cur); ++k, ++done) {
+    const int nb = cur.nb;
+    // the next unit's Q, K_0 and V_0 are fetched into L2 a few ring units
+    // before this unit ends, so its first loads need not wait for HBM
+    const int pf_at = max(0, nb - 3);
+    for (int u = 0; u <= nb; ++u, ++ug) {
+      const int us = ug % C::kUnits;
+      const uint32_t ph = (ug / C::kUnits) & 1;
+      const uint32_t bar_full = bars + 8u * (1 + us);
+      const uint32_t bar_empty = bars + 8u * (1 + C::kStages + us);
+      if (!(ok = wait_one(bar_empty, ph ^ 1u, wd))) break;
+      const bool has_v = u >= 1;
+      const bool has_k = u < nb;
+      mbar_arrive_expect_tx(bar_full, (int(has_v) + int(has_k)) * C::kTileBytes);
+      if (has_v) {
 #pragma unroll
-  for (int g = 0; g < 2; ++g)
+        for (int a = 0; a < C::kAtoms; ++a)
+          tma_load_3d_hint(sRing + (2 * us) * C::kTileBytes + a * C::kAtomBytes, tv, bar_full,
+                           a * 64, (u - 1) * kTileRows, cur.bh, pol_kv);
+      }
+      if (has_k) {
 #pragma unroll
-    for (int a = 0; a < C::kAtoms; ++a)
-      tma_load_3d_hint(sQ + g * C::kTileBytes + a * C::kAtomBytes, tq, bar_q, a * 64,
-                       q0 + g * kTileRows, bh, pol_q);
-
-  // K/V arrive in units that the MMA warp consumes together: unit 0 = K_0,
-  // unit u >= 1 = (V_{u-1}, K_u), the last unit V only. A unit occupies two
-  // tile slots of the ring (V in the first, K in the second) and has one full
-  // and one empty barrier, so the MMA warp waits once per step for its tiles.
-  const int n_units = n_kv_b + 1;
-  int u = 0;
-  for (; u < n_units; ++u) {
-    const int us = u % C::kUnits;
-    const uint32_t ph = (u / C::kUnits) & 1;
-    const uint32_t bar_full = bars + 8u * (1 + us);
-    const uint32_t bar_empty = bars + 8u * (1 + C::kStages + us);
-    if (!wait_one(bar_empty, ph ^ 1u, wd)) break;
-    const bool has_v = u >= 1;
-    const bool has_k = u < n_kv_b;
-    mbar_arrive_expect_tx(bar_full, (int(has_v) + int(has_k)) * C::kTileBytes);
-    if (has_v) {
+        for (int a = 0; a < C::kAtoms; ++a)
+          tma_load_3d_hint(sRing + (2 * us + 1) * C::kTileBytes + a * C::kAtomBytes, tk, bar_full,
+                           a * 64, u * kTileRows, cur.bh, pol_kv);
+      }
+      if (u == 0) {
+        if (done > 0 && !(ok = wait_one(bar_q_empty, (done - 1) & 1, wd))) break;
+        mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
 #pragma unroll
-      for (int a = 0; a < C::kAtoms; ++a)
-        tma_load_3d_hint(sRing + (2 * us) * C::kTileBytes + a * C::kAtomBytes, tv, bar_full,
-                         a * 64, (u - 1) * kTileRows, bh, pol_kv);
-    }
-    if (has_k) {
+        for (int g = 0; g < 2; ++g)
 #pragma unroll
-      for (int a = 0; a < C::kAtoms; ++a)
-        tma_load_3d_hint(sRing + (2 * us + 1) * C::kTileBytes + a * C::kAtomBytes, tk, bar_full,
-                         a * 64, u * kTileRows, bh, pol_kv);
+          for (int a = 0; a < C::kAtoms; ++a)
+            tma_load_3d_hint(sQ + g * C::kTileBytes + a * C::kAtomBytes, tq, bar_q, a * 64,
+                             cur.q0 + g * kTileRows, cur.bh, pol_q);
+      }
+      if (u == pf_at) {
+        int k2 = k + 1;
+        SquareUnit nxt;
+        if (square_unit(p, k2, nxt)) {
+#pragma unroll
+          for (int a = 0; a < C::kAtoms; ++a) {
+            tma_prefetch_l2_3d(tq, a * 64, nxt.q0, nxt.bh);
+            tma_prefetch_l2_3d(tq, a * 64, nxt.q0 + kTileRows, nxt.bh);
+            tma_prefetch_l2_3d(tk, a * 64, 0, nxt.bh);
+            tma_prefetch_l2_3d(tv, a * 64, 0, nxt.bh);
+          }
+        }
+      }
     }
   }
   // Teardown: every copy this thread issued must have landed before exit.
-  drain_wait(bar_q, 0, wd);
-  for (int w = (u > C::kUnits ? u - C::kUnits : 0); w < u; ++w)
+  if (done > 0) drain_wait(bar_q, (done - 1) & 1, wd);
+  for (int w = (ug > C::kUnits ? ug - C::kUnits : 0); w < ug; ++w)
     drain_wait(bars + 8u * (1 + w % C::kUnits), (w / C::kUnits) & 1, wd);
 }
 
 template <int D, bool kF8 = false>
-__device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t bars, int na,
-                                         int nb, uint32_t qk_negate, const Watchdog& wd) {
+__device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t bars,
+                                         const FwdParams& p, const Watchdog& wd) {
+  const uint32_t qk_negate = p.qk_negate;
   using C = Cfg<D, kF8>;
   const uint32_t sQ = base + C::kQOff;
   const uint32_t sRing = base + C::kRingOff;
@@ -628,7 +725,10 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   const uint32_t v_lo = static_cast<uint32_t>(sdesc_sw128(sRing, C::kAtomBytes, 1024));
   auto mk = [&](uint32_t lo) { return kk_hi | lo; };
   auto issue_qk = [&](int g, int slot) {
-    const uint32_t a0 = q_lo + static_cast<uint32_t>((g * C::kTileBytes) >> 4);
+    // the opaque move keeps the compiler from hoisting every Q descriptor of
+    // the unit loop into registers (the issuing warp has few to spare)
+    uint32_t a0;
+    asm volatile("mov.b32 %0, %1;" : "=r"(a0) : "r"(q_lo + static_cast<uint32_t>((g * C::kTileBytes) >> 4)));
     const uint32_t b0 = r_lo + static_cast<uint32_t>((slot * C::kTileBytes) >> 4);
 #pragma unroll
     for (int kk = 0; kk < D / C::kMmaK; ++kk) {
@@ -656,39 +756,51 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
     }
   };
 
-  bool ok = wait_one(bar_q, 0, wd) && wait_one(full_bar(0), par_of(0), wd);
-  if (ok) {
+  const uint32_t bar_q_empty = bar_s_full0 + 56u;
+  int ug = 0;                // ring position, across work units
+  uint32_t pa = 0, pb = 0;   // P hand-offs of tile a / b taken so far
+  int done = 0;              // work units of this CTA so far
+  bool ok = true;
+  SquareUnit cur;
+  for (int k = 0; ok && square_unit(p, k, cur); ++k, ++done) {
+    const int na = cur.na, nb = cur.nb;
+    if (!(ok = wait_one(bar_q, done & 1, wd) && wait_one(full_bar(ug), par_of(ug), wd))) break;
     tc_fence_after_sync();
-    issue_qk(0, k_slot(0));
+    issue_qk(0, k_slot(ug));
     mma_commit(bar_s_full0);
-    issue_qk(1, k_slot(0));
+    issue_qk(1, k_slot(ug));
     mma_commit(bar_s_full0 + 8u);
-    mma_commit(empty_bar(0));
-  }
-  for (int j = 0; ok && j < nb; ++j) {
-    const int u = j + 1;  // V_j and K_{j+1}
-    if (!(ok = wait_one(full_bar(u), par_of(u), wd))) break;
-    if (j < na) {
-      if (!(ok = wait_spin(bar_p_ready0, j & 1, wd))) break;
-      tc_fence_after_sync();
-      issue_pv(0, v_slot(u), j > 0);
-      if (j + 1 < na) {
-        issue_qk(0, k_slot(u));
-        mma_commit(bar_s_full0);
-      } else {
-        mma_commit(bar_o_final0);
+    if (nb == 1) mma_commit(bar_q_empty);  // the unit's last Q K^T
+    mma_commit(empty_bar(ug));
+    ++ug;
+    for (int j = 0; j < nb; ++j, ++ug) {
+      // ring unit ug: V_j and K_{j+1}
+      if (!(ok = wait_one(full_bar(ug), par_of(ug), wd))) break;
+      if (j < na) {
+        if (!(ok = wait_spin(bar_p_ready0, pa & 1, wd))) break;
+        ++pa;
+        tc_fence_after_sync();
+        issue_pv(0, v_slot(ug), j > 0);
+        if (j + 1 < na) {
+          issue_qk(0, k_slot(ug));
+          mma_commit(bar_s_full0);
+        } else {
+          mma_commit(bar_o_final0);
+        }
       }
+      if (!(ok = wait_spin(bar_p_ready0 + 8u, pb & 1, wd))) break;
+      ++pb;
+      tc_fence_after_sync();
+      issue_pv(1, v_slot(ug), j > 0);
+      if (j + 1 < nb) {
+        issue_qk(1, k_slot(ug));
+        mma_commit(bar_s_full0 + 8u);
+        if (j + 2 == nb) mma_commit(bar_q_empty);  // the unit's last Q K^T
+      } else {
+        mma_commit(bar_o_final0 + 8u);
+      }
+      mma_commit(empty_bar(ug));
     }
-    if (!(ok = wait_spin(bar_p_ready0 + 8u, j & 1, wd))) break;
-    tc_fence_after_sync();
-    issue_pv(1, v_slot(u), j > 0);
-    if (j + 1 < nb) {
-      issue_qk(1, k_slot(u));
-      mma_commit(bar_s_full0 + 8u);
-    } else {
-      mma_commit(bar_o_final0 + 8u);
-    }
-    mma_commit(empty_bar(u));
   }
   // Teardown: all MMAs this thread issued must be complete before the tensor
   // memory is freed.
@@ -887,7 +999,8 @@ template <int D, bool kKV, bool kF8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                           const __grid_constant__ CUtensorMap tmap_k,
-                          const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
+                          const __grid_constant__ CUtensorMap tmap_v,
+                          const __grid_constant__ CUtensorMap tmap_o, const FwdParams p) {
   static_assert(!(kKV && kF8), "the FP8 path covers the square problem");
   using C = Cfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
@@ -901,18 +1014,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32;
   const uint32_t lane = threadIdx.x % 32;
 
-  // Work unit: heads are the slow index so co-resident CTAs share K/V in L2;
-  // with causal masking the heaviest query blocks go first.
-  int bh, q0, na, nb;
+  // Work: the kv path's CTA is one (head, key range, query block); a square
+  // path CTA walks the work units blockIdx.x, blockIdx.x + gridDim.x, ...
+  // (square_unit), one after another on the same barriers and buffers.
+  int bh = 0, q0 = 0, na = 0, nb = 0;
   KvWork kw{0, 0, 0, 0};
-  if constexpr (!kKV) {
-    bh = blockIdx.x / p.nqb;
-    const int r = blockIdx.x % p.nqb;
-    const int qblk = p.causal ? (p.nqb - 1 - r) : r;
-    q0 = qblk * kBlockRows;
-    na = p.causal ? min(p.T, q0 / kTileRows + 1) : p.T;
-    nb = p.causal ? min(p.T, q0 / kTileRows + 2) : p.T;
-  } else {
+  if constexpr (kKV) {
     kw = kv_work_of(p, bh, q0);
     na = kw.na;
     nb = kw.nb;
@@ -932,6 +1039,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(b6 + 32, 1);   // o_final a
     mbar_init(b6 + 40, 1);   // o_final b
     mbar_init(b6 + 48, 1);   // mma_done
+    mbar_init(b6 + 56, 1);   // q_empty
+    mbar_init(b6 + 64, 1);   // stage_free
     *abort_flag = 0u;
     mbar_fence_init();
   }
@@ -939,6 +1048,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
+    if constexpr (!kKV) tma_prefetch_desc(&tmap_o);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -951,18 +1061,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Watchdog wd{abort_flag, p.err, p.wait_limit_ns};
 
   if (warp < 8) {
-    regs_increase<kRegsSoftmax>();
+    regs_increase<kRegsSoftmax<kKV>>();
     const int g = warp / 4;
-    softmax_role<D, kKV, kF8>(p, tmem, bars + 8u * (1 + 2 * C::kStages), bh, q0,
-                              g == 0 ? na : nb, g, wd, kw.kv_lo);
+    const uint32_t ctl = bars + 8u * (1 + 2 * C::kStages);
+    if constexpr (kKV) {
+      softmax_role<D, kKV, kF8>(p, tmem, ctl, bh, q0, g == 0 ? na : nb, g, wd, kw.kv_lo);
+    } else {
+      uint32_t steps = 0;  // this warpgroup's S hand-offs so far (s_full phases)
+      uint32_t done = 0;   // work units so far (o_final phases)
+      SquareUnit u;
+      for (int k = 0; square_unit(p, k, u); ++k, ++done) {
+        const int n = g == 0 ? u.na : u.nb;
+        if (!softmax_role<D, kKV, kF8>(p, tmem, ctl, u.bh, u.q0, n, g, wd, 0, steps, done & 1,
+                                       &tmap_o, base + C::kStageOff, 2 * done + g))
+          break;
+        steps += n;
+      }
+      // the O stores this warpgroup's leader issued complete before exit
+      if (threadIdx.x % 128 == 0) bulk_wait_all();
+    }
   } else {
-    regs_decrease<kRegsOther>();
+    regs_decrease<kRegsOther<kKV>>();
     if constexpr (!kKV) {
       if (warp == kProducerWarp) {
-        if (lane == 0)
-          producer_role<D, kF8>(&tmap_q, &tmap_k, &tmap_v, base, bars, bh, q0, nb, wd);
+        if (lane == 0) producer_role<D, kF8>(&tmap_q, &tmap_k, &tmap_v, base, bars, p, wd);
       } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_role<D, kF8>(tmem, base, bars, na, nb, p.qk_negate, wd);
+        if (lane == 0) mma_role<D, kF8>(tmem, base, bars, p, wd);
       }
     } else {
       const bool alt = p.alt != 0;
@@ -1103,6 +1227,19 @@ unsigned int* device_error_word() {
   return ptr;
 }
 
+// Multiprocessors of the current device, cached per context.
+int sm_count_current() {
+  static CtxCache<int> cache;
+  int n = 0;
+  if (!cache.get(&n, [](int* out) {
+        int dev = 0;
+        return cudaGetDevice(&dev) == cudaSuccess &&
+               cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
+      }))
+    return 0;
+  return n;
+}
+
 // Once per (kernel, context): raise the kernel's dynamic shared-memory limit
 // and check the register allocation the in-kernel register split relies on
 // (the softmax warpgroups' setmaxnreg increase draws on exactly the launch
@@ -1134,9 +1271,11 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0
   using C = Cfg<D, kF8>;
   const int BH = a.B * a.H;
   CUtensorMap mq, mk, mv;
+  CUtensorMap mo;
   if (!encode_qkv_map(&mq, a.q, BH, a.N, D, C::kElemBytes) ||
       !encode_qkv_map(&mk, a.k, BH, a.N, D, C::kElemBytes) ||
-      !encode_qkv_map(&mv, a.v, BH, a.N, D, C::kElemBytes))
+      !encode_qkv_map(&mv, a.v, BH, a.N, D, C::kElemBytes) ||
+      !encode_qkv_map(&mo, a.o, BH, a.N, D, 2))
     return ATTN_ERR_CUDA;
   unsigned int* err = device_error_word();
   if (!err) return ATTN_ERR_CUDA;
@@ -1154,12 +1293,16 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0
   p.v_descale = v_descale;
   p.causal = a.causal;
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-  const long long grid = static_cast<long long>(p.nqb) * BH;
-  if (grid > 0x7fffffffLL) return ATTN_ERR_SHAPE;
+  const long long units = static_cast<long long>(p.nqb) * BH;
+  if (units > 0x7fffffffLL) return ATTN_ERR_SHAPE;
   const int prep = prepare_kernel<fused_attn_fwd_kernel<D, false, kF8>>(C::kSmemBytes);
   if (prep != ATTN_OK) return prep;
+  // persistent grid: one CTA per SM (one fits), each walking work units
+  const int sms = sm_count_current();
+  if (sms < 1) return ATTN_ERR_CUDA;
+  const long long grid = std::min<long long>(units, sms);
   fused_attn_fwd_kernel<D, false, kF8>
-      <<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+      <<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
@@ -1208,7 +1351,7 @@ int launch_fused_kv_d(const AttnKvArgs& a, const KvPlan& plan, void* workspace,
   const int prep = prepare_kernel<fused_attn_fwd_kernel<D, true>>(C::kSmemBytesKv);
   if (prep != ATTN_OK) return prep;
   fused_attn_fwd_kernel<D, true>
-      <<<static_cast<unsigned>(grid), kThreads, C::kSmemBytesKv, stream>>>(mq, mk, mv, p);
+      <<<static_cast<unsigned>(grid), kThreads, C::kSmemBytesKv, stream>>>(mq, mk, mv, mv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   if (plan.nsplit > 1)
     return launch_lse_combine(p.part_o, p.part_lse, a.o, a.lse, BH * a.Nq, D, plan.nsplit, stream);
