@@ -140,31 +140,79 @@ def profiled_kv_traffic(w):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    """SM clock, power and clock-event reasons sampled every 5 ms by an NVML
+    thread while the timed region runs (a 20-step region lasts ~70 ms, too
+    short for nvidia-smi's 200 ms loop). Falls back to nvidia-smi at its
+    shortest interval when NVML cannot be loaded. Reads settings only."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.005
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:  # noqa: BLE001 - any lookup failure: fall back to the index
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _nvml_loop(self, nv, h, stop):
+        sm_max = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+        while not stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mw = nv.nvmlDeviceGetPowerUsage(h)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:  # noqa: BLE001 - a failed read ends sampling
+                break
+            self.rows.append([str(self.gpu), str(sm), str(sm_max), f"{mw / 1000:.1f}", hex(r)]
+                             + ["Active" if r & b else "Not Active" for b in bits])
+            stop.wait(self.PERIOD_S)
 
     def __enter__(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, self.stop),
+                                           daemon=True)
+            self.thread.start()
+            self.source = f"nvml every {self.PERIOD_S * 1e3:.0f} ms"
+            return self
+        except Exception:  # noqa: BLE001 - no NVML: nvidia-smi below
+            self.thread = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi every 20 ms"
         except (OSError, FileNotFoundError):
             self.proc = None
         time.sleep(0.3)
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -173,14 +221,16 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        rows = []
+        rows = list(self.rows)
         if self.path and os.path.exists(self.path):
             for line in open(self.path):
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) >= 9:
                     rows.append(parts)
             os.unlink(self.path)
-        return summarize_clocks(rows)
+        out = summarize_clocks(rows)
+        out["source"] = self.source
+        return out
 
 
 def summarize_clocks(rows):
@@ -199,8 +249,11 @@ def summarize_clocks(rows):
         for name, val in zip(names, r[5:9]):
             if val.strip().lower() == "active":
                 reasons.add(name)
+    watts = [num(r[3]) for r in rows if num(r[3]) is not None]
     return {"sm_mhz": statistics.median(sm) if sm else None,
             "sm_max_mhz": max(mx) if mx else None,
+            "sm_mhz_min": min(sm) if sm else None,
+            "power_w_median": statistics.median(watts) if watts else None,
             "reasons": sorted(reasons), "samples": len(rows)}
 
 
@@ -468,7 +521,8 @@ def run_ours(args):
         barrier(dist)
     ms_local = start.elapsed_time(end)
     bounds = [start, *marks, end]
-    per_step = sorted(a.elapsed_time(b) for a, b in zip(bounds[:-1], bounds[1:]))
+    in_order = [a.elapsed_time(b) for a, b in zip(bounds[:-1], bounds[1:])]
+    per_step = sorted(in_order)
     ms_total = max_over_ranks(ms_local, dist, device)
     if ea.last_device_error() != 0:
         raise SystemExit("device watchdog fired in the timed region")
@@ -500,6 +554,7 @@ def run_ours(args):
         "ms_per_step": ms_step,
         "ms_per_step_median_rank0": statistics.median(per_step),
         "ms_per_step_best_rank0": per_step[0],
+        "ms_per_step_in_order_rank0": [round(t, 4) for t in in_order],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,

@@ -59,7 +59,8 @@ def test_workloads_all_rows(name):
     w = WORKLOADS[name]
     q, k, v = make_workload(w)
     o, lse = _run(q, k, v, w.scale, w.causal)
-    check_against_oracle(q, k, v, o, lse, w.scale, w.causal, what=name)
+    e = check_against_oracle(q, k, v, o, lse, w.scale, w.causal, what=name)
+    print(name, e)
 
 
 @pytest.mark.parametrize("name", ["long_8192_causal", "stress_65536_causal"])

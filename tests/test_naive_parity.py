@@ -47,15 +47,17 @@ def test_bert_base_all_rows():
     w = WORKLOADS["bert_base_1024"]
     q, k, v = make_workload(w)
     o, lse = _run(q, k, v, w.scale, w.causal)
-    check_naive_against_oracle(q, k, v, o, lse, w.scale, w.causal, what="naive bert")
+    e = check_naive_against_oracle(q, k, v, o, lse, w.scale, w.causal, what="naive bert")
+    print("naive", w.name, e)
 
 
 def test_decoder_sampled():
     w = WORKLOADS["decoder_2048_causal"]
     q, k, v = make_workload(w)
     o, lse = _run(q, k, v, w.scale, w.causal)
-    check_naive_against_oracle(q, k, v, o, lse, w.scale, w.causal, rows=sampled(w),
-                               what="naive dec")
+    e = check_naive_against_oracle(q, k, v, o, lse, w.scale, w.causal, rows=sampled(w),
+                                   what="naive dec")
+    print("naive", w.name, e)
 
 
 def test_naive_and_fused_agree():
