@@ -250,10 +250,12 @@ def summarize_clocks(rows):
             if val.strip().lower() == "active":
                 reasons.add(name)
     watts = [num(r[3]) for r in rows if num(r[3]) is not None]
+    masks = sorted({r[4] for r in rows if r[4].startswith("0x")})
     return {"sm_mhz": statistics.median(sm) if sm else None,
             "sm_max_mhz": max(mx) if mx else None,
             "sm_mhz_min": min(sm) if sm else None,
             "power_w_median": statistics.median(watts) if watts else None,
+            "reason_masks": masks,
             "reasons": sorted(reasons), "samples": len(rows)}
 
 
@@ -581,7 +583,9 @@ def run_ours(args):
             "algorithmic_bytes": costs.fused_bytes(w.B, w.H, w.N, w.d),
             "kernel": "fused_attn_fwd_kernel<128, false, false>",
         },
-        "clocks": {k: clock_info[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "clocks": {k: clock_info.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "sm_mhz_min",
+                                                  "power_w_median", "reason_masks", "samples",
+                                                  "source")},
         "e2e": e2e,
         "gpu_launches": args.steps,
     }
