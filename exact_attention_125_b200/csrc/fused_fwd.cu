@@ -100,17 +100,18 @@ constexpr float kBiasBoundSlack = 96.0f;
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 
 // Which of a row's 64 (even, odd) column pairs take the FMA-pipe exponential
-// (exp2_poly_pair) instead of the MUFU one. bf16: three pairs in eight (2, 5
-// and 7 of every eight), which took ~14 % off a tile's softmax arithmetic
-// against one in four, with the row sum moved after the P hand-off. FP8: the
-// E4M3 MMAs take half the bf16 time, so the softmax is the longer leg by far
-// and the FMA pipe has room for one pair in three (measured: 1/3 beats 1/4 by
-// 4 % and 1/2 is slower than both).
+// (exp2_poly_pair) instead of the MUFU one. bf16: one pair in four. Measured
+// on the persistent kernel at (8, 32, 8192, 128, causal): 1/4 is 1 % faster
+// than 3/8 below the power cap and 0.5 % under it, all-MUFU lies between,
+// 1/2 is 5 % slower. FP8: the E4M3 MMAs take half the bf16 time, so the
+// softmax is the longer leg by far and the FMA pipe has room for one pair in
+// three (measured on the one-CTA-per-unit kernel: 1/3 beats 1/4 by 4 % and
+// 1/2 is slower than both).
 constexpr int kPolyPeriodF8 = 3;
 template <bool kF8>
 __host__ __device__ constexpr bool poly_pair(int cc) {
   if constexpr (kF8) return cc % kPolyPeriodF8 == kPolyPeriodF8 - 1;
-  return (cc % 8) == 2 || (cc % 8) == 5 || (cc % 8) == 7;
+  return (cc % 4) == 3;
 }
 
 // kF8: Q, K, V hold 8-bit E4M3 values (one byte each) instead of bf16.
