@@ -940,7 +940,9 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
             "window_left": wl, "window_right": wr, "distance_bias": bias, "num_splits": splits,
             "ms_per_step": ms, "steps": steps, "tflops": tf, "bound": "tensor",
             "peak_tflops": float(peaks["bf16_tflops"]), "frac": tf / float(peaks["bf16_tflops"]),
-            "kernel": "fused_attn_fwd_kernel<128, true, false>"}
+            "kernel": ("fused_attn_fwd_kernel<128, false, false> (square problem, unsplit)"
+                       if Nq == Nk and wl < 0 and wr < 0 and splits == 1
+                       else "fused_attn_fwd_kernel<128, true, false>")}
 
 
 def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):

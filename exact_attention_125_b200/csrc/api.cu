@@ -146,6 +146,24 @@ int fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, in
     if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   }
   if ((st = check_device()) != ATTN_OK) return st;
+  if (Nq == Nk && window_left < 0 && window_right < 0 && plan.nsplit == 1) {
+    // the square problem, unsplit: the persistent square kernel, which takes
+    // the distance bias too (the workspace stays unused)
+    attn::AttnArgs s;
+    s.q = q;
+    s.k = k;
+    s.v = v;
+    s.o = o;
+    s.lse = lse;
+    s.B = B;
+    s.H = H;
+    s.N = Nq;
+    s.d = d;
+    s.scale = scale;
+    s.causal = causal;
+    s.slopes = slopes;
+    return attn::launch_fused(s, reinterpret_cast<cudaStream_t>(stream));
+  }
   attn::AttnKvArgs a;
   a.q = q;
   a.k = k;

@@ -292,8 +292,10 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
     key_lo = lo_of(row);
     tile_hi = hi_of(row_start);
     tile_lo = lo_of(row_start + kTileRows - 1);
-    if (p.slopes) slope_l2 = p.slopes[bh % p.H] * 1.4426950408889634f;
   }
+  if (p.slopes) slope_l2 = p.slopes[bh % p.H] * 1.4426950408889634f;
+  // sequence position of query row 0 (keys start at position 0)
+  const int pos_offset = kKV ? p.offset : 0;
 
   float m_run = -INFINITY;
   float l_run = 0.0f;
@@ -307,9 +309,9 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
     bool need_mask;
     int col0;
     float cs = c;  // multiplier from the values in sr to log2-domain logits
-    // kv path, distance bias on a tile wholly on one side of every row's
-    // position: b(cc) = bias_b0 + bias_dk * cc (log2 units), applied in the
-    // exponent rather than to sr
+    // distance bias on a tile wholly on one side of every row's position:
+    // b(cc) = bias_b0 + bias_dk * cc (log2 units), applied in the exponent
+    // rather than to sr
     bool bias_linear = false;
     float bias_b0 = 0.0f, bias_dk = 0.0f;
     if constexpr (kKV) {
@@ -322,27 +324,6 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
         for (int cc = 0; cc < 128; ++cc)
           sr[cc] = (cc > lim_hi || cc < lim_lo) ? 0xff800000u : (zero_scale ? 0u : sr[cc]);  // -inf
       }
-      if (p.slopes) {
-        // linear distance bias: x = s * c - slope * log2(e) * |pos - key|
-        const float rel = static_cast<float>(row + p.offset - col0);  // pos - col0
-        const bool left = col0 + kTileRows - 1 <= row_start + p.offset;   // key <= pos everywhere
-        const bool right = col0 >= row_start + kTileRows - 1 + p.offset;  // key >= pos everywhere
-        if ((left || right) && slope_l2 * (kTileRows - 1) <= kBiasBoundSlack) {
-          // One side of every row's position: the bias is linear in the
-          // column, b(cc) = b0 + dk * cc. The scores stay unbiased here; the
-          // row maximum is bounded by max(s) * c + max(b) and the bias enters
-          // the exponent's FMA (below), one packed add per pair.
-          bias_dk = left ? slope_l2 : -slope_l2;
-          bias_b0 = -bias_dk * rel;
-          bias_linear = true;
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 128; ++cc)
-            sr[cc] = __float_as_uint(
-                fmaf(__uint_as_float(sr[cc]), c, -slope_l2 * fabsf(rel - static_cast<float>(cc))));
-          cs = 1.0f;  // sr now holds the biased log2-domain logits
-        }
-      }
     } else {
       col0 = j * kTileRows;
       need_mask =
@@ -353,6 +334,27 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc)
           sr[cc] = cc > lim ? 0xff800000u : (zero_scale ? 0u : sr[cc]);  // -inf
+      }
+    }
+    if (p.slopes) {
+      // linear distance bias: x = s * c - slope * log2(e) * |pos - key|
+      const float rel = static_cast<float>(row + pos_offset - col0);  // pos - col0
+      const bool left = col0 + kTileRows - 1 <= row_start + pos_offset;   // key <= pos everywhere
+      const bool right = col0 >= row_start + kTileRows - 1 + pos_offset;  // key >= pos everywhere
+      if ((left || right) && slope_l2 * (kTileRows - 1) <= kBiasBoundSlack) {
+        // One side of every row's position: the bias is linear in the
+        // column, b(cc) = b0 + dk * cc. The scores stay unbiased here; the
+        // row maximum is bounded by max(s) * c + max(b) and the bias enters
+        // the exponent's FMA (below), one packed add per pair.
+        bias_dk = left ? slope_l2 : -slope_l2;
+        bias_b0 = -bias_dk * rel;
+        bias_linear = true;
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 128; ++cc)
+          sr[cc] = __float_as_uint(
+              fmaf(__uint_as_float(sr[cc]), c, -slope_l2 * fabsf(rel - static_cast<float>(cc))));
+        cs = 1.0f;  // sr now holds the biased log2-domain logits
       }
     }
 
@@ -1294,6 +1296,8 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0
   p.v_descale = v_descale;
   p.causal = a.causal;
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  p.H = a.H;
+  p.slopes = a.slopes;
   const long long units = static_cast<long long>(p.nqb) * BH;
   if (units > 0x7fffffffLL) return ATTN_ERR_SHAPE;
   const int prep = prepare_kernel<fused_attn_fwd_kernel<D, false, kF8>>(C::kSmemBytes);

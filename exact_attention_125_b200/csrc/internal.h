@@ -18,6 +18,8 @@ struct AttnArgs {
   int B, H, N, d;
   float scale;
   int causal;
+  // per-head linear distance bias slopes (natural-log units), or null
+  const float* slopes = nullptr;
 };
 
 // Fused tcgen05 path (fused_fwd.cu). Arguments already validated.

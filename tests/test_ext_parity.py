@@ -31,6 +31,12 @@ CASES = [
     (1, 2, 700, 700, 128, True, 255, -1, "steep", 0),
     (1, 1, 300, 200, 64, False, 10, 10, None, 1),   # early rows: no key in their window
     (1, 3, 17, 4096, 64, True, 511, -1, "alibi", 0),
+    # square problems without a window run on the persistent square kernel:
+    # non-causal (tiles left of, right of and across the diagonal), steep
+    # slopes (the bias added per logit), d = 64, ragged N
+    (1, 2, 300, 300, 128, False, -1, -1, "alibi", 1),
+    (1, 2, 513, 513, 64, True, -1, -1, "steep", 0),
+    (2, 2, 384, 384, 128, False, -1, -1, "steep", 1),
 ]
 
 
@@ -52,6 +58,7 @@ def test_ext_all_rows(B, H, Nq, Nk, d, causal, wl, wr, kind, splits):
     (1, 2, 300, 300, 128, True, 63, -1, "alibi", 1),
     (1, 2, 100, 1100, 128, True, 300, -1, None, 4),
     (1, 4, 1, 3000, 64, False, -1, -1, "alibi", 3),
+    (1, 2, 300, 300, 128, True, -1, -1, "alibi", 1),
 ])
 def test_ext_zero_and_negative_scale(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale):
     _ext_case(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale)
@@ -89,6 +96,17 @@ def test_ext_without_options_matches_attn_fwd_kv_bit_for_bit():
     qg, kg, vg = (t.to("cuda") for t in (q, k, v))
     o1, l1 = ea.attn_fwd_kv(qg, kg, vg, causal=True, num_splits=3)
     o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=True, num_splits=3)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_square_ext_without_options_matches_attn_fwd_bit_for_bit(causal):
+    # Nq == Nk, no window, no bias: the square kernel serves both entry points
+    q, k, v = make_q_kv(1, 3, 700, 700, 128, seed=11 + int(causal))
+    qg, kg, vg = (t.to("cuda") for t in (q, k, v))
+    o1, l1 = ea.attn_fwd(qg, kg, vg, causal=causal)
+    o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=causal, num_splits=1)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
