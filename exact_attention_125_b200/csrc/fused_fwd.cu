@@ -247,7 +247,7 @@ __device__ __forceinline__ void store_row_chunk(const FwdParams& p, bool partial
 // s_phase0: steps this warpgroup has taken before (the square path's work
 // units follow one another on the same barriers); o_phase: parity of this
 // unit's o_final phase. Returns false once a wait has given up.
-template <int D, bool kKV, bool kF8 = false>
+template <int D, bool kKV, bool kF8 = false, bool kBias = kKV>
 __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, uint32_t ctl,
                                              int bh, int q0, int n_kv, int g,
                                              const Watchdog& wd, int kv_lo, uint32_t s_phase0 = 0,
@@ -293,7 +293,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
     tile_hi = hi_of(row_start);
     tile_lo = lo_of(row_start + kTileRows - 1);
   }
-  if (p.slopes) slope_l2 = p.slopes[bh % p.H] * 1.4426950408889634f;
+  if (kBias && p.slopes) slope_l2 = p.slopes[bh % p.H] * 1.4426950408889634f;
   // sequence position of query row 0 (keys start at position 0)
   const int pos_offset = kKV ? p.offset : 0;
 
@@ -336,7 +336,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
           sr[cc] = cc > lim ? 0xff800000u : (zero_scale ? 0u : sr[cc]);  // -inf
       }
     }
-    if (p.slopes) {
+    if (kBias && p.slopes) {
       // linear distance bias: x = s * c - slope * log2(e) * |pos - key|
       const float rel = static_cast<float>(row + pos_offset - col0);  // pos - col0
       const bool left = col0 + kTileRows - 1 <= row_start + pos_offset;   // key <= pos everywhere
@@ -998,7 +998,7 @@ __device__ __forceinline__ void mma_role_kv(uint32_t tmem, uint32_t base, uint32
 // kD: head dimension. kKV: the kv path (Nq query rows against N keys, the
 // KV range of each head split across CTAs); false: the square problem.
 // kF8 (square problem only): E4M3 Q, K, V and P.
-template <int D, bool kKV, bool kF8 = false>
+template <int D, bool kKV, bool kF8 = false, bool kBias = kKV>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                           const __grid_constant__ CUtensorMap tmap_k,
@@ -1068,14 +1068,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = warp / 4;
     const uint32_t ctl = bars + 8u * (1 + 2 * C::kStages);
     if constexpr (kKV) {
-      softmax_role<D, kKV, kF8>(p, tmem, ctl, bh, q0, g == 0 ? na : nb, g, wd, kw.kv_lo);
+      softmax_role<D, kKV, kF8, kBias>(p, tmem, ctl, bh, q0, g == 0 ? na : nb, g, wd, kw.kv_lo);
     } else {
       uint32_t steps = 0;  // this warpgroup's S hand-offs so far (s_full phases)
       uint32_t done = 0;   // work units so far (o_final phases)
       SquareUnit u;
       for (int k = 0; square_unit(p, k, u); ++k, ++done) {
         const int n = g == 0 ? u.na : u.nb;
-        if (!softmax_role<D, kKV, kF8>(p, tmem, ctl, u.bh, u.q0, n, g, wd, 0, steps, done & 1,
+        if (!softmax_role<D, kKV, kF8, kBias>(p, tmem, ctl, u.bh, u.q0, n, g, wd, 0, steps, done & 1,
                                        &tmap_o, base + C::kStageOff, 2 * done + g))
           break;
         steps += n;
@@ -1300,14 +1300,19 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0
   p.slopes = a.slopes;
   const long long units = static_cast<long long>(p.nqb) * BH;
   if (units > 0x7fffffffLL) return ATTN_ERR_SHAPE;
-  const int prep = prepare_kernel<fused_attn_fwd_kernel<D, false, kF8>>(C::kSmemBytes);
+  // the distance bias has an instantiation of its own, so that the plain
+  // kernel's exponent loop carries no bias arithmetic
+  constexpr auto plain = fused_attn_fwd_kernel<D, false, kF8, false>;
+  constexpr auto biased = fused_attn_fwd_kernel<D, false, kF8, !kF8>;
+  const bool use_bias = !kF8 && a.slopes != nullptr;
+  const int prep = use_bias ? prepare_kernel<biased>(C::kSmemBytes) : prepare_kernel<plain>(C::kSmemBytes);
   if (prep != ATTN_OK) return prep;
   // persistent grid: one CTA per SM (one fits), each walking work units
   const int sms = sm_count_current();
   if (sms < 1) return ATTN_ERR_CUDA;
   const long long grid = std::min<long long>(units, sms);
-  fused_attn_fwd_kernel<D, false, kF8>
-      <<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+  (use_bias ? biased : plain)<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
+      mq, mk, mv, mo, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
