@@ -613,12 +613,12 @@ __device__ __forceinline__ bool square_unit(const FwdParams& p, int& k, SquareUn
   }
 }
 
-// Square path producer: for each of the CTA's work units, the K/V units of
-// its KV tiles (unit 0 = K_0, unit u >= 1 = (V_{u-1}, K_u), the last V only)
-// into the ring, which runs on across work units, and the unit's two Q tiles
-// once the previous unit's last Q K^T has completed (q_empty). K_0 of the next
-// unit is requested before that wait, so both arrive while the current unit's
-// last step is still running.
+// Square path producer. The ring runs on across the CTA's work units: ring
+// unit 0 holds K_0 of the first unit; for each unit, ring units 1..nb hold
+// (V_{u-1}, K_u), and its last one holds V_{nb-1} with K_0 of the next unit
+// in the otherwise empty K half, so the next unit's first Q K^T needs no
+// ring unit of its own. The next unit's Q tiles are loaded once the current
+// unit's last Q K^T has completed (q_empty).
 template <int D, bool kF8 = false>
 __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUtensorMap* tk,
                                               const CUtensorMap* tv, uint32_t base, uint32_t bars,
@@ -630,50 +630,53 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
   const uint32_t bar_q_empty = bars + 8u * (1 + 2 * C::kStages + 7);
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  int ug = 0;    // ring position, across work units
+  auto load_tile = [&](int slot, const CUtensorMap* map, int row, int bh, uint32_t bar_full) {
+#pragma unroll
+    for (int a = 0; a < C::kAtoms; ++a)
+      tma_load_3d_hint(sRing + slot * C::kTileBytes + a * C::kAtomBytes, map, bar_full, a * 64, row, bh,
+                       pol_kv);
+  };
+  auto load_q = [&](const SquareUnit& u) {
+    mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+      for (int a = 0; a < C::kAtoms; ++a)
+        tma_load_3d_hint(sQ + g * C::kTileBytes + a * C::kAtomBytes, tq, bar_q, a * 64,
+                         u.q0 + g * kTileRows, u.bh, pol_q);
+  };
+  // fills ring unit ug with the given tiles (row < 0: none) once its slot is free
+  auto fill = [&](int ug, int v_row, int v_bh, int k_row, int k_bh) -> bool {
+    const int us = ug % C::kUnits;
+    const uint32_t bar_full = bars + 8u * (1 + us);
+    if (!wait_one(bars + 8u * (1 + C::kStages + us), ((ug / C::kUnits) & 1) ^ 1u, wd)) return false;
+    mbar_arrive_expect_tx(bar_full, (int(v_row >= 0) + int(k_row >= 0)) * C::kTileBytes);
+    if (v_row >= 0) load_tile(2 * us, tv, v_row, v_bh, bar_full);
+    if (k_row >= 0) load_tile(2 * us + 1, tk, k_row, k_bh, bar_full);
+    return true;
+  };
+  int ug = 0;    // ring units filled so far
   int done = 0;  // work units of this CTA so far
   bool ok = true;
+  int k = 0;
   SquareUnit cur;
-  for (int k = 0; ok && square_unit(p, k, cur); ++k, ++done) {
-    const int nb = cur.nb;
-    // the next unit's Q, K_0 and V_0 are fetched into L2 a few ring units
-    // before this unit ends, so its first loads need not wait for HBM
-    const int pf_at = max(0, nb - 3);
-    for (int u = 0; u <= nb; ++u, ++ug) {
-      const int us = ug % C::kUnits;
-      const uint32_t ph = (ug / C::kUnits) & 1;
-      const uint32_t bar_full = bars + 8u * (1 + us);
-      const uint32_t bar_empty = bars + 8u * (1 + C::kStages + us);
-      if (!(ok = wait_one(bar_empty, ph ^ 1u, wd))) break;
-      const bool has_v = u >= 1;
-      const bool has_k = u < nb;
-      mbar_arrive_expect_tx(bar_full, (int(has_v) + int(has_k)) * C::kTileBytes);
-      if (has_v) {
-#pragma unroll
-        for (int a = 0; a < C::kAtoms; ++a)
-          tma_load_3d_hint(sRing + (2 * us) * C::kTileBytes + a * C::kAtomBytes, tv, bar_full,
-                           a * 64, (u - 1) * kTileRows, cur.bh, pol_kv);
-      }
-      if (has_k) {
-#pragma unroll
-        for (int a = 0; a < C::kAtoms; ++a)
-          tma_load_3d_hint(sRing + (2 * us + 1) * C::kTileBytes + a * C::kAtomBytes, tk, bar_full,
-                           a * 64, u * kTileRows, cur.bh, pol_kv);
-      }
-      if (u == 0) {
-        if (done > 0 && !(ok = wait_one(bar_q_empty, (done - 1) & 1, wd))) break;
-        mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
-#pragma unroll
-        for (int g = 0; g < 2; ++g)
-#pragma unroll
-          for (int a = 0; a < C::kAtoms; ++a)
-            tma_load_3d_hint(sQ + g * C::kTileBytes + a * C::kAtomBytes, tq, bar_q, a * 64,
-                             cur.q0 + g * kTileRows, cur.bh, pol_q);
-      }
-      if (u == pf_at) {
-        int k2 = k + 1;
-        SquareUnit nxt;
-        if (square_unit(p, k2, nxt)) {
+  if (square_unit(p, k, cur)) {
+    ok = fill(ug++, -1, 0, 0, cur.bh);  // K_0 of the first unit
+    if (ok) load_q(cur);
+    while (ok) {
+      int k2 = k + 1;
+      SquareUnit nxt{0, 0, 0, 0};
+      const bool has_next = square_unit(p, k2, nxt);
+      const int nb = cur.nb;
+      // the next unit's Q, K_0 and V_0 are fetched into L2 a few ring units
+      // before this unit ends, so its first loads need not wait for HBM
+      const int pf_at = max(1, nb - 3);
+      for (int u = 1; ok && u <= nb; ++u) {
+        if (u < nb)
+          ok = fill(ug++, (u - 1) * kTileRows, cur.bh, u * kTileRows, cur.bh);
+        else
+          ok = fill(ug++, (u - 1) * kTileRows, cur.bh, has_next ? 0 : -1, nxt.bh);
+        if (ok && u == pf_at && has_next) {
 #pragma unroll
           for (int a = 0; a < C::kAtoms; ++a) {
             tma_prefetch_l2_3d(tq, a * 64, nxt.q0, nxt.bh);
@@ -683,6 +686,13 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
           }
         }
       }
+      ++done;
+      if (!ok || !has_next) break;
+      // the next unit's Q once this unit's last Q K^T has completed
+      if (!(ok = wait_one(bar_q_empty, (done - 1) & 1, wd))) break;
+      load_q(nxt);
+      k = k2;
+      cur = nxt;
     }
   }
   // Teardown: every copy this thread issued must have landed before exit.
@@ -760,50 +770,90 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   };
 
   const uint32_t bar_q_empty = bar_s_full0 + 56u;
-  int ug = 0;                // ring position, across work units
+  int ug = 0;                // ring unit holding K_0 of the current work unit
   uint32_t pa = 0, pb = 0;   // P hand-offs of tile a / b taken so far
   int done = 0;              // work units of this CTA so far
+  bool early_a = false;      // S_a(0) of the current unit already issued
   bool ok = true;
+  int k = 0;
   SquareUnit cur;
-  for (int k = 0; ok && square_unit(p, k, cur); ++k, ++done) {
+  bool have = square_unit(p, k, cur);
+  while (ok && have) {
     const int na = cur.na, nb = cur.nb;
+    int k2 = k + 1;
+    SquareUnit nxt;
+    const bool has_next = square_unit(p, k2, nxt);
     if (!(ok = wait_one(bar_q, done & 1, wd) && wait_one(full_bar(ug), par_of(ug), wd))) break;
     tc_fence_after_sync();
-    issue_qk(0, k_slot(ug));
-    mma_commit(bar_s_full0);
+    if (!early_a) {
+      issue_qk(0, k_slot(ug));
+      mma_commit(bar_s_full0);
+    }
     issue_qk(1, k_slot(ug));
     mma_commit(bar_s_full0 + 8u);
     if (nb == 1) mma_commit(bar_q_empty);  // the unit's last Q K^T
+    // ring unit ug: K_0 (and the previous unit's last V): read by now
     mma_commit(empty_bar(ug));
-    ++ug;
-    for (int j = 0; j < nb; ++j, ++ug) {
-      // ring unit ug: V_j and K_{j+1}
-      if (!(ok = wait_one(full_bar(ug), par_of(ug), wd))) break;
+    early_a = false;
+    for (int j = 0; j < nb; ++j) {
+      const int ru = ug + j + 1;  // V_j, and K_{j+1} (the last: K_0 of the next unit)
+      if (!(ok = wait_one(full_bar(ru), par_of(ru), wd))) break;
       if (j < na) {
         if (!(ok = wait_spin(bar_p_ready0, pa & 1, wd))) break;
         ++pa;
         tc_fence_after_sync();
-        issue_pv(0, v_slot(ug), j > 0);
+        issue_pv(0, v_slot(ru), j > 0);
         if (j + 1 < na) {
-          issue_qk(0, k_slot(ug));
+          issue_qk(0, k_slot(ru));
           mma_commit(bar_s_full0);
         } else {
           mma_commit(bar_o_final0);
         }
       }
+      if (j + 1 == nb && has_next) {
+        // tile b's last P is still being computed: tile a's first Q K^T of the
+        // next unit goes as soon as the next Q tiles land, so that tile a's
+        // softmax starts that unit while tile b finishes this one
+        uint64_t t0 = 0;
+        for (uint32_t it = 1;; ++it) {
+          if (mbar_test_wait(bar_p_ready0 + 8u, pb & 1)) break;
+          if (mbar_test_wait(bar_q, (done + 1) & 1)) {
+            tc_fence_after_sync();
+            issue_qk(0, k_slot(ru));
+            mma_commit(bar_s_full0);
+            early_a = true;
+            break;
+          }
+          if ((it & 63) == 0) {
+            if (t0 == 0) t0 = global_timer_ns();
+            if (*wd.abort || timed_out(t0, wd)) {
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (!ok) break;
+      }
       if (!(ok = wait_spin(bar_p_ready0 + 8u, pb & 1, wd))) break;
       ++pb;
       tc_fence_after_sync();
-      issue_pv(1, v_slot(ug), j > 0);
+      issue_pv(1, v_slot(ru), j > 0);
       if (j + 1 < nb) {
-        issue_qk(1, k_slot(ug));
+        issue_qk(1, k_slot(ru));
         mma_commit(bar_s_full0 + 8u);
         if (j + 2 == nb) mma_commit(bar_q_empty);  // the unit's last Q K^T
       } else {
         mma_commit(bar_o_final0 + 8u);
       }
-      mma_commit(empty_bar(ug));
+      // the last ring unit also holds the next unit's K_0: released after
+      // that unit's first Q K^T
+      if (j + 1 < nb || !has_next) mma_commit(empty_bar(ru));
     }
+    ug += nb;
+    ++done;
+    k = k2;
+    cur = nxt;
+    have = has_next;
   }
   // Teardown: all MMAs this thread issued must be complete before the tensor
   // memory is freed.
