@@ -161,6 +161,9 @@ struct FwdParams {
   // when scale < 0, so the softmax always multiplies by a positive factor
   uint32_t qk_negate;
   int causal;
+  // square path: 1 when the work units are dealt in (heaviest, lightest)
+  // pairs (more units than CTAs); 0: one unit per CTA
+  int paired;
   uint64_t wait_limit_ns;
   // kv path only (Nq query rows against N keys, KV range split across CTAs)
   int Nq;
@@ -588,13 +591,24 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
 // counter, and pairs are head-major so the CTAs running at the same time share
 // K/V in L2. Unit k of the CTA is half k % 2 of its pair k / 2 (the heavy
 // block first); with nqb odd the middle block of a head forms a pair alone.
-// Every role of the CTA walks the same sequence.
+// With no more units than SMs (p.paired = 0) each CTA takes the one unit
+// blockIdx.x instead. Every role of the CTA walks the same sequence.
 struct SquareUnit {
   int bh, q0, na, nb;
 };
 
 // k: the CTA's unit index, advanced past a skipped (absent) second half.
 __device__ __forceinline__ bool square_unit(const FwdParams& p, int& k, SquareUnit& u) {
+  if (!p.paired) {
+    // one wave: unit blockIdx.x alone
+    if (k > 0 || static_cast<int>(blockIdx.x) >= p.nqb * p.BH) return false;
+    u.bh = blockIdx.x / p.nqb;
+    const int r = blockIdx.x % p.nqb;
+    u.q0 = (p.causal ? p.nqb - 1 - r : r) * kBlockRows;
+    u.na = p.causal ? min(p.T, u.q0 / kTileRows + 1) : p.T;
+    u.nb = p.causal ? min(p.T, u.q0 / kTileRows + 2) : p.T;
+    return true;
+  }
   const int npairs = (p.nqb + 1) / 2;
   while (true) {
     const int pair = static_cast<int>(blockIdx.x) + (k / 2) * static_cast<int>(gridDim.x);
@@ -1357,9 +1371,12 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0
   const bool use_bias = !kF8 && a.slopes != nullptr;
   const int prep = use_bias ? prepare_kernel<biased>(C::kSmemBytes) : prepare_kernel<plain>(C::kSmemBytes);
   if (prep != ATTN_OK) return prep;
-  // persistent grid: one CTA per SM (one fits), each walking work units
+  // persistent grid: one CTA per SM (one fits), each walking work units in
+  // balanced pairs; with no more units than SMs, one unit per CTA (pairing
+  // would only put two units behind each other on half the CTAs)
   const int sms = sm_count_current();
   if (sms < 1) return ATTN_ERR_CUDA;
+  p.paired = units > sms ? 1 : 0;
   const long long grid = std::min<long long>(units, sms);
   (use_bias ? biased : plain)<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
       mq, mk, mv, mo, p);
