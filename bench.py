@@ -169,28 +169,34 @@ class ClockSampler:
         except Exception:  # noqa: BLE001 - any lookup failure: fall back to the index
             return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
-    def _nvml_loop(self, nv, h, stop):
-        sm_max = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+    def _nvml_sample(self):
+        nv, h = self.nv, self.handle
         bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
                 nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
-        while not stop.is_set():
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                mw = nv.nvmlDeviceGetPowerUsage(h)
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-            except Exception:  # noqa: BLE001 - a failed read ends sampling
-                break
-            self.rows.append([str(self.gpu), str(sm), str(sm_max), f"{mw / 1000:.1f}", hex(r)]
-                             + ["Active" if r & b else "Not Active" for b in bits])
-            stop.wait(self.PERIOD_S)
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:  # noqa: BLE001 - a failed read is skipped
+            return
+        try:
+            watts = f"{nv.nvmlDeviceGetPowerUsage(h) / 1000:.1f}"
+        except Exception:  # noqa: BLE001 - power is optional
+            watts = "n/a"
+        self.rows.append([str(self.gpu), str(sm), str(self.sm_max), watts, hex(r)]
+                         + ["Active" if r & b else "Not Active" for b in bits])
+
+    def _nvml_loop(self, stop):
+        while not stop.wait(self.PERIOD_S):
+            self._nvml_sample()
 
     def __enter__(self):
         import threading
         try:
-            nv, h = self._nvml_handle()
+            self.nv, self.handle = self._nvml_handle()
+            self.sm_max = self.nv.nvmlDeviceGetMaxClockInfo(self.handle, self.nv.NVML_CLOCK_SM)
+            self._nvml_sample()  # one sample as the timed region starts, whatever the thread does
             self.stop = threading.Event()
-            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, self.stop),
-                                           daemon=True)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(self.stop,), daemon=True)
             self.thread.start()
             self.source = f"nvml every {self.PERIOD_S * 1e3:.0f} ms"
             return self
@@ -213,6 +219,7 @@ class ClockSampler:
         if self.thread is not None:
             self.stop.set()
             self.thread.join(timeout=5)
+            self._nvml_sample()  # and one as it ends
         if self.proc is not None:
             self.proc.terminate()
             try:
