@@ -56,7 +56,9 @@ def _check(q8, k8, v8, ds, scale, causal, rows, o, lse, what):
 
 
 @pytest.mark.parametrize("B,H,N,causal", [(1, 2, 300, False), (1, 2, 300, True), (2, 3, 1000, True),
-                                          (1, 1, 129, False), (1, 1, 1, True), (1, 2, 640, False)])
+                                          (1, 1, 129, False), (1, 1, 1, True), (1, 2, 640, False),
+                                          # more 256-row units than SMs: dealt in pairs
+                                          (1, 80, 700, True)])
 def test_fp8_small_all_rows(B, H, N, causal):
     (q8, k8, v8), ds = make_qkv_fp8(B, H, N, 128, seed=N + 5 * int(causal))
     o, lse = ea.attn_fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), *ds, scale=128 ** -0.5, causal=causal)

@@ -47,6 +47,26 @@ def _run(q, k, v, scale, causal):
     return o, lse
 
 
+# Enough (batch, head) pairs that the 256-row work units outnumber the SMs,
+# so the persistent kernel deals them to its CTAs in (heaviest, lightest)
+# pairs across several units per CTA, carrying each next unit's first K tile
+# in the previous unit's last ring unit; an odd number of blocks per head (the
+# middle block forms a pair alone) and a ragged last block.
+MANY_UNITS = [
+    # B, H, N, d, causal
+    (2, 40, 700, 128, True),
+    (2, 40, 700, 64, False),
+    (1, 80, 1100, 128, True),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", MANY_UNITS)
+def test_many_units_odd_blocks_all_rows(B, H, N, d, causal):
+    q, k, v = make_qkv(B, H, N, d, seed=3 * N + d + int(causal))
+    o, lse = _run(q, k, v, scale_of(d), causal)
+    check_against_oracle(q, k, v, o, lse, scale_of(d), causal, what=f"{(B, H, N, d, causal)}")
+
+
 @pytest.mark.parametrize("B,H,N,d,causal", SMALL)
 def test_small_shapes_all_rows(B, H, N, d, causal):
     q, k, v = make_qkv(B, H, N, d, seed=N * 7 + d + int(causal))
