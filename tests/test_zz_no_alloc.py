@@ -7,8 +7,9 @@ cudaMalloc/cudaFree would add a device-wide synchronisation. For them the
 library keeps S and P in its own fixed device array. This test calls that
 entry point through the C ABI twice in a row, on different inputs, and checks
 each result against attn_fwd_naive with a caller-owned workspace, using the
-tolerances of the other parity tests. The file is named so that pytest
-collects it last.
+tolerances of the other parity tests, and against the fp64 oracle with the
+unfused path's derived bound. The file is named so that pytest collects it
+last.
 """
 import numpy as np
 import pytest
@@ -63,6 +64,17 @@ def test_no_alloc_matches_workspace_path_twice(B, H, N, d, causal):
     for call, seed in enumerate((100 + N, 200 + N)):
         q, k, v = (t.cuda() for t in make_qkv(B, H, N, d, seed=seed))
         _close(_with_workspace(q, k, v, scale, causal), _no_alloc(q, k, v, scale, causal))
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", [(1, 2, 1000, 64, True), (2, 1, 333, 128, False)])
+def test_no_alloc_against_the_oracle(B, H, N, d, causal):
+    # the same bound the workspace path is held to (bf16 S, derived allowance)
+    from parity_util import check_naive_against_oracle
+    scale = 1.0 / float(np.sqrt(d))
+    q, k, v = make_qkv(B, H, N, d, seed=300 + N + int(causal))
+    o, lse = _no_alloc(q.cuda(), k.cuda(), v.cuda(), scale, causal)
+    torch.cuda.synchronize()
+    check_naive_against_oracle(q, k, v, o, lse, scale, causal, what=f"noalloc {(B, H, N, d, causal)}")
 
 
 def test_no_alloc_rejects_sizes_over_the_limit():
