@@ -80,13 +80,13 @@ constexpr int kMmaWarp = 9;     // warps 10 and 11 only give their registers awa
 // host refuses to launch otherwise), and the split after setmaxnreg. The
 // split uses exactly the launch total.
 constexpr int kRegsAtLaunch = 168;
-// kv path: 224 for each softmax warpgroup, 56 for the producer/MMA one; the
-// persistent square path gives the producer and MMA warps 88 for their work
-// loop (its softmax fits in 208).
+// Both paths: 216 for each softmax warpgroup, 72 for the producer/MMA one
+// (the split-KV instantiation spilled more with 224/56: 52 bytes against 8 at
+// d = 128, and ran 1 % slower).
 template <bool kKV>
-constexpr int kRegsSoftmax = kKV ? 224 : 216;
+constexpr int kRegsSoftmax = 216;
 template <bool kKV>
-constexpr int kRegsOther = kKV ? 56 : 72;
+constexpr int kRegsOther = 72;
 static_assert(128 * (2 * kRegsSoftmax<true> + kRegsOther<true>) == kThreads * kRegsAtLaunch &&
                   128 * (2 * kRegsSoftmax<false> + kRegsOther<false>) == kThreads * kRegsAtLaunch,
               "register split must equal the launch allocation");
