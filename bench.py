@@ -23,6 +23,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -84,11 +85,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C++ source without its comments and trailing blanks: what the compiler
+    turns into code (string literals in these sources hold no comment
+    markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def source_hash(paths=None) -> str:
+    """Hash of the kernel sources' code (comments left out), which gates the
+    committed ncu traffic figures: a comment edit leaves them valid, any code
+    edit voids them."""
     h = hashlib.sha256()
     for path in (paths or KERNEL_SOURCES):
-        with open(path, "rb") as f:
-            h.update(f.read())
+        with open(path, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -9,15 +9,19 @@
 // tiling and fusion, never touch HBM": tiles plus a running softmax
 // normalisation, one kernel, HBM paid once).
 //
-// Work unit: one (batch*head, block of 256 query rows) per CTA, split into two
+// Work unit: one (batch*head, block of 256 query rows), split into two
 // 128-row query tiles "a" and "b" that ping-pong: while the softmax warps of
-// one tile turn S into P, the tensor core runs the other tile's MMAs.
+// one tile turn S into P, the tensor core runs the other tile's MMAs. The
+// square problem runs a persistent grid: one CTA per SM walks its work units
+// (square_unit) on the same barriers and buffers, starting each unit's loads
+// while the previous one finishes.
 //
 // Roles (384 threads):
 //   warps 0-3  softmax + epilogue of query tile a (thread t owns row t)
 //   warps 4-7  softmax + epilogue of query tile b
-//   warp  8    TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... into
-//              a ring of shared-memory stages (128B-swizzled, mbarrier-tracked)
+//   warp  8    TMA producer: Q tiles, then K_0, (V_0, K_1), (V_1, K_2), ...
+//              into a ring of shared-memory stages (128B-swizzled,
+//              mbarrier-tracked)
 //   warp  9    tensor-memory allocator and single-thread tcgen05 MMA issuer
 //   warps 10-11 only hand their registers to the softmax warps (setmaxnreg)
 //
@@ -32,7 +36,8 @@
 //
 // The FP8 instantiation (kF8 = true, square problem, d = 128) takes E4M3 Q,
 // K, V, runs both products as tcgen05 kind::f8f6f4 MMAs and stores P as four
-// E4M3 values per tensor-memory column (32 columns).
+// E4M3 values per tensor-memory column (32 columns). The kBias instantiation
+// of the square problem adds the per-head linear distance bias.
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_a [0,128), S_b [128,256),
 // O_a [256, 256+d), O_b [256+d, 256+2d). P (bf16, two per column) overwrites
