@@ -97,6 +97,16 @@ def test_profiled_traffic_is_gated_by_source_hash_and_workload(tmp_path, monkeyp
     assert bench.profiled_traffic("long_8192_causal") is None
 
 
+def test_source_hash_follows_code_not_comments(tmp_path):
+    src = tmp_path / "k.cu"
+    src.write_text("// header\nint f(int x) {  /* doubled */\n  return 2 * x;  // twice\n}\n")
+    h0 = bench.source_hash([str(src)])
+    src.write_text("// another header\n\nint f(int x) {\n  return 2 * x;\n}\n/* trailing\n   note */\n")
+    assert bench.source_hash([str(src)]) == h0  # comments and blank lines only
+    src.write_text("int f(int x) {\n  return 3 * x;\n}\n")
+    assert bench.source_hash([str(src)]) != h0  # a code edit
+
+
 def test_bench_arguments_parse():
     a = bench.parse_args(["--gpus", "2", "--steps", "3", "--warmup", "4", "--no-naive",
                           "--no-kv", "--no-ext", "--no-chain", "--no-fp8"])
