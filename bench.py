@@ -842,7 +842,7 @@ def host_overhead_line(device, n_calls=2000):
     ts.sort()
     return {"workload": w.name, "calls": n_calls, "us_median": ts[len(ts) // 2] / 1e3,
             "us_p10": ts[len(ts) // 10] / 1e3, "us_p90": ts[9 * len(ts) // 10] / 1e3,
-            "includes": "Python ctypes call, validation, three tensor-map encodings, launch"}
+            "includes": "Python ctypes call, validation, four tensor-map encodings, launch"}
 
 
 KV_BENCH_WORKLOADS = ("decode_131072", "chunk_128x32768_causal")
