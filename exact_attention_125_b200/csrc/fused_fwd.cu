@@ -1316,7 +1316,7 @@ int sm_count_current() {
 // and check the register allocation the in-kernel register split relies on
 // (the softmax warpgroups' setmaxnreg increase draws on exactly the launch
 // allocation, so any other count could make it wait forever; the build also
-// rejects such a binary). Later calls in the same context reuse the verdict.
+// rejects such a binary). Later calls in the same context reuse that result.
 template <auto Kernel>
 int prepare_kernel(int smem_bytes) {
   static CtxCache<int> cache;
