@@ -113,3 +113,37 @@ def test_bench_arguments_parse():
     assert (a.gpus, a.steps, a.warmup, a.impl) == (2, 3, 4, "ours")
     assert a.no_naive and a.no_kv and a.no_ext and a.no_chain and a.no_fp8
     assert bench.parse_args(["--impl", "reference"]).impl == "reference"
+
+
+def test_clock_sampler_reads_nvml_inside_the_region(monkeypatch):
+    # a fake NVML: the SM clock drops and the power-cap reason appears after
+    # a few reads, as under a long load on a 1 kW part
+    import sys
+    import types
+    calls = {"n": 0}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0,
+        nvmlClocksEventReasonHwSlowdown=0x8, nvmlClocksEventReasonHwThermalSlowdown=0x40,
+        nvmlClocksEventReasonSwThermalSlowdown=0x20, nvmlClocksEventReasonSwPowerCap=0x4,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByUUID=lambda uuid: "h",
+        nvmlDeviceGetHandleByIndex=lambda i: "h",
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965)
+
+    def clock(h, c):
+        calls["n"] += 1
+        return 1965 if calls["n"] < 4 else 1560
+
+    fake.nvmlDeviceGetClockInfo = clock
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x0 if calls["n"] < 4 else 0x4
+    fake.nvmlDeviceGetPowerUsage = lambda h: 990000
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    import time
+    sampler = bench.ClockSampler(0)
+    with sampler:
+        time.sleep(0.05)
+    s = sampler.summary()
+    assert s["samples"] >= 2 and s["source"].startswith("nvml")
+    assert s["sm_max_mhz"] == 1965.0 and s["sm_mhz_min"] == 1560.0
+    assert "sw_power_cap" in s["reasons"] and "hw_slowdown" not in s["reasons"]
+    assert s["power_w_median"] == 990.0
