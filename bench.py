@@ -601,7 +601,7 @@ def run_ours(args):
             "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peaks_kind}, burst)",
             "traffic": profiled_traffic(w.name),
             "algorithmic_bytes": costs.fused_bytes(w.B, w.H, w.N, w.d),
-            "kernel": "fused_attn_fwd_kernel<128, false, false>",
+            "kernel": "fused_attn_fwd_kernel<128, false, false, false, false>",
         },
         "clocks": {k: clock_info.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "sm_mhz_min",
                                                   "power_w_median", "reason_masks", "samples",
@@ -900,8 +900,8 @@ def split_kv_line(name, device, peaks, steps=10, warmup=3):
             "frac_of_datasheet_7700": gbs / HBM_DATASHEET_GBS,
             "above_measured_copy_peak": gbs > float(peaks["hbm_gbs"]),
             "bound": "hbm", "traffic": profiled_kv_traffic(w),
-            "kernel": "fused_attn_fwd_kernel<128, true, false>" + (" + lse_combine_kernel<128>"
-                                                            if splits > 1 else ""),
+            "kernel": "fused_attn_fwd_kernel<128, true, false, true, false>" + (
+                " + lse_combine_kernel<128>" if splits > 1 else ""),
             "tflops": flops / (ms * 1e-3) / 1e12,
             "launches_per_step": 2 if splits > 1 else 1,
             "l2": "inputs larger than L2"}
@@ -960,9 +960,10 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
             "window_left": wl, "window_right": wr, "distance_bias": bias, "num_splits": splits,
             "ms_per_step": ms, "steps": steps, "tflops": tf, "bound": "tensor",
             "peak_tflops": float(peaks["bf16_tflops"]), "frac": tf / float(peaks["bf16_tflops"]),
-            "kernel": ("fused_attn_fwd_kernel<128, false, false> (square problem, unsplit)"
-                       if Nq == Nk and wl < 0 and wr < 0 and splits == 1
-                       else "fused_attn_fwd_kernel<128, true, false>")}
+            "kernel": (f"fused_attn_fwd_kernel<128, false, false, {str(bool(bias)).lower()}, "
+                       f"{str(wl >= 0 or wr >= 0).lower()}> (square problem, unsplit)"
+                       if Nq == Nk and splits == 1
+                       else "fused_attn_fwd_kernel<128, true, false, true, false>")}
 
 
 def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
@@ -1045,7 +1046,7 @@ def fp8_line(w, device, peaks, steps=10, warmup=3):
             "tflops": tf, "bound": "tensor", "peak_tflops": peak,
             "peak_source": "2 x MEASURED_PEAKS.json bf16_tflops (nominal FP8 / bf16 ratio)",
             "frac": tf / peak, "speedup_over_bf16_line": None,
-            "kernel": "fused_attn_fwd_kernel<128, false, true>"}
+            "kernel": "fused_attn_fwd_kernel<128, false, true, false, false>"}
 
 
 def main(argv=None):

@@ -146,9 +146,9 @@ int fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, in
     if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   }
   if ((st = check_device()) != ATTN_OK) return st;
-  if (Nq == Nk && window_left < 0 && window_right < 0 && plan.nsplit == 1) {
+  if (Nq == Nk && plan.nsplit == 1) {
     // the square problem, unsplit: the persistent square kernel, which takes
-    // the distance bias too (the workspace stays unused)
+    // the key windows and the distance bias too (the workspace stays unused)
     attn::AttnArgs s;
     s.q = q;
     s.k = k;
@@ -162,6 +162,8 @@ int fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, in
     s.scale = scale;
     s.causal = causal;
     s.slopes = slopes;
+    s.window_left = window_left;
+    s.window_right = window_right;
     return attn::launch_fused(s, reinterpret_cast<cudaStream_t>(stream));
   }
   attn::AttnKvArgs a;

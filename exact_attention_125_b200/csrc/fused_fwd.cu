@@ -37,7 +37,9 @@
 // The FP8 instantiation (kF8 = true, square problem, d = 128) takes E4M3 Q,
 // K, V, runs both products as tcgen05 kind::f8f6f4 MMAs and stores P as four
 // E4M3 values per tensor-memory column (32 columns). The kBias instantiation
-// of the square problem adds the per-head linear distance bias.
+// of the square problem adds the per-head linear distance bias, and the kWin
+// one applies key windows: each work unit starts at the KV tile of its first
+// row's first key and ends at its last row's last one.
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_a [0,128), S_b [128,256),
 // O_a [256, 256+d), O_b [256+d, 256+2d). P (bf16, two per column) overwrites
@@ -251,11 +253,12 @@ __device__ __forceinline__ void store_row_chunk(const FwdParams& p, bool partial
 }
 
 // ctl: shared address of the control barriers s_full[2], p_ready[2],
-// o_final[2] (consecutive).
+// o_final[2] (consecutive). kWin (square path): per-row key ranges as on the
+// kv path, KV tiles counted from kv_lo.
 // s_phase0: steps this warpgroup has taken before (the square path's work
 // units follow one another on the same barriers); o_phase: parity of this
 // unit's o_final phase. Returns false once a wait has given up.
-template <int D, bool kKV, bool kF8 = false, bool kBias = kKV>
+template <int D, bool kKV, bool kF8 = false, bool kBias = kKV, bool kWin = false>
 __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, uint32_t ctl,
                                              int bh, int q0, int n_kv, int g,
                                              const Watchdog& wd, int kv_lo, uint32_t s_phase0 = 0,
@@ -279,12 +282,14 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
   // scaled by 1 (scaling -inf by 0 would give NaN)
   const bool zero_scale = p.scale_log2 == 0.0f;
   const float c = zero_scale ? 1.0f : p.scale_log2;
-  // kv path: this row's allowed keys [key_lo, key_hi] (causal limit, window,
-  // key count); the tile's first row has the lowest key_hi and its last row
-  // the highest key_lo, which decide whether a KV tile needs masking at all.
+  // kv path and windows: this row's allowed keys [key_lo, key_hi] (causal
+  // limit, window, key count); the tile's first row has the lowest key_hi and
+  // its last row the highest key_lo, which decide whether a KV tile needs
+  // masking at all.
+  constexpr bool kRange = kKV || kWin;
   int key_lo = 0, key_hi = p.N - 1, tile_hi = p.N - 1, tile_lo = 0;
   float slope_l2 = 0.0f;
-  if constexpr (kKV) {
+  if constexpr (kRange) {
     auto hi_of = [&](int r) {
       long long h = p.N - 1;
       if (p.causal) h = min(h, static_cast<long long>(r) + p.offset);
@@ -322,7 +327,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
     // rather than to sr
     bool bias_linear = false;
     float bias_b0 = 0.0f, bias_dk = 0.0f;
-    if constexpr (kKV) {
+    if constexpr (kRange) {
       col0 = (kv_lo + (alt ? 2 * j + g : j)) * kTileRows;
       need_mask = (col0 + kTileRows - 1 > tile_hi) || (col0 < tile_lo) || zero_scale;
       if (need_mask) {
@@ -598,11 +603,38 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
 // block first); with nqb odd the middle block of a head forms a pair alone.
 // With no more units than SMs (p.paired = 0) each CTA takes the one unit
 // blockIdx.x instead. Every role of the CTA walks the same sequence.
+// With a key window (kWin) a unit starts at KV tile j0, the tile of the first
+// key its first row may see, and na / nb count tiles from there; without one
+// j0 = 0.
 struct SquareUnit {
-  int bh, q0, na, nb;
+  int bh, q0, na, nb, j0;
 };
 
+// The KV tiles of the unit at q0: [j0, j0 + na) for query tile a and
+// [j0, j0 + nb) for tile b (nb - na is 0 or 1).
+template <bool kWin>
+__device__ __forceinline__ void square_range(const FwdParams& p, SquareUnit& u) {
+  if constexpr (kWin) {
+    // one past the last KV tile that row r sees (causal limit, right window
+    // bound, key count)
+    auto end_of = [&](int r) {
+      long long hi = p.N - 1;
+      if (p.causal) hi = min(hi, static_cast<long long>(r));
+      if (p.wr >= 0) hi = min(hi, static_cast<long long>(r) + p.wr);
+      return static_cast<int>(hi / kTileRows) + 1;
+    };
+    u.j0 = (p.wl >= 0 ? max(0, u.q0 - p.wl) : 0) / kTileRows;
+    u.na = end_of(u.q0 + kTileRows - 1) - u.j0;
+    u.nb = end_of(u.q0 + kBlockRows - 1) - u.j0;
+  } else {
+    u.j0 = 0;
+    u.na = p.causal ? min(p.T, u.q0 / kTileRows + 1) : p.T;
+    u.nb = p.causal ? min(p.T, u.q0 / kTileRows + 2) : p.T;
+  }
+}
+
 // k: the CTA's unit index, advanced past a skipped (absent) second half.
+template <bool kWin = false>
 __device__ __forceinline__ bool square_unit(const FwdParams& p, int& k, SquareUnit& u) {
   if (!p.paired) {
     // one wave: unit blockIdx.x alone
@@ -610,8 +642,7 @@ __device__ __forceinline__ bool square_unit(const FwdParams& p, int& k, SquareUn
     u.bh = blockIdx.x / p.nqb;
     const int r = blockIdx.x % p.nqb;
     u.q0 = (p.causal ? p.nqb - 1 - r : r) * kBlockRows;
-    u.na = p.causal ? min(p.T, u.q0 / kTileRows + 1) : p.T;
-    u.nb = p.causal ? min(p.T, u.q0 / kTileRows + 2) : p.T;
+    square_range<kWin>(p, u);
     return true;
   }
   const int npairs = (p.nqb + 1) / 2;
@@ -626,8 +657,7 @@ __device__ __forceinline__ bool square_unit(const FwdParams& p, int& k, SquareUn
     }
     u.bh = pair / npairs;
     u.q0 = qblk * kBlockRows;
-    u.na = p.causal ? min(p.T, u.q0 / kTileRows + 1) : p.T;
-    u.nb = p.causal ? min(p.T, u.q0 / kTileRows + 2) : p.T;
+    square_range<kWin>(p, u);
     return true;
   }
 }
@@ -637,8 +667,9 @@ __device__ __forceinline__ bool square_unit(const FwdParams& p, int& k, SquareUn
 // (V_{u-1}, K_u), and its last one holds V_{nb-1} with K_0 of the next unit
 // in the otherwise empty K half, so the next unit's first Q K^T needs no
 // ring unit of its own. The next unit's Q tiles are loaded once the current
-// unit's last Q K^T has completed (q_empty).
-template <int D, bool kF8 = false>
+// unit's last Q K^T has completed (q_empty). Tile indices count from the
+// unit's j0.
+template <int D, bool kF8 = false, bool kWin = false>
 __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUtensorMap* tk,
                                               const CUtensorMap* tv, uint32_t base, uint32_t bars,
                                               const FwdParams& p, const Watchdog& wd) {
@@ -679,29 +710,32 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
   bool ok = true;
   int k = 0;
   SquareUnit cur;
-  if (square_unit(p, k, cur)) {
-    ok = fill(ug++, -1, 0, 0, cur.bh);  // K_0 of the first unit
+  // first key row of a unit
+  auto key0 = [](const SquareUnit& u) { return kWin ? u.j0 * kTileRows : 0; };
+  if (square_unit<kWin>(p, k, cur)) {
+    ok = fill(ug++, -1, 0, key0(cur), cur.bh);  // K_0 of the first unit
     if (ok) load_q(cur);
     while (ok) {
       int k2 = k + 1;
-      SquareUnit nxt{0, 0, 0, 0};
-      const bool has_next = square_unit(p, k2, nxt);
+      SquareUnit nxt{0, 0, 0, 0, 0};
+      const bool has_next = square_unit<kWin>(p, k2, nxt);
       const int nb = cur.nb;
+      const int r0 = key0(cur);
       // the next unit's Q, K_0 and V_0 are fetched into L2 a few ring units
       // before this unit ends, so its first loads need not wait for HBM
       const int pf_at = max(1, nb - 3);
       for (int u = 1; ok && u <= nb; ++u) {
         if (u < nb)
-          ok = fill(ug++, (u - 1) * kTileRows, cur.bh, u * kTileRows, cur.bh);
+          ok = fill(ug++, r0 + (u - 1) * kTileRows, cur.bh, r0 + u * kTileRows, cur.bh);
         else
-          ok = fill(ug++, (u - 1) * kTileRows, cur.bh, has_next ? 0 : -1, nxt.bh);
+          ok = fill(ug++, r0 + (u - 1) * kTileRows, cur.bh, has_next ? key0(nxt) : -1, nxt.bh);
         if (ok && u == pf_at && has_next) {
 #pragma unroll
           for (int a = 0; a < C::kAtoms; ++a) {
             tma_prefetch_l2_3d(tq, a * 64, nxt.q0, nxt.bh);
             tma_prefetch_l2_3d(tq, a * 64, nxt.q0 + kTileRows, nxt.bh);
-            tma_prefetch_l2_3d(tk, a * 64, 0, nxt.bh);
-            tma_prefetch_l2_3d(tv, a * 64, 0, nxt.bh);
+            tma_prefetch_l2_3d(tk, a * 64, key0(nxt), nxt.bh);
+            tma_prefetch_l2_3d(tv, a * 64, key0(nxt), nxt.bh);
           }
         }
       }
@@ -720,7 +754,7 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tq, const CUten
     drain_wait(bars + 8u * (1 + w % C::kUnits), (w / C::kUnits) & 1, wd);
 }
 
-template <int D, bool kF8 = false>
+template <int D, bool kF8 = false, bool kWin = false>
 __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t bars,
                                          const FwdParams& p, const Watchdog& wd) {
   const uint32_t qk_negate = p.qk_negate;
@@ -796,12 +830,12 @@ __device__ __forceinline__ void mma_role(uint32_t tmem, uint32_t base, uint32_t 
   bool ok = true;
   int k = 0;
   SquareUnit cur;
-  bool have = square_unit(p, k, cur);
+  bool have = square_unit<kWin>(p, k, cur);
   while (ok && have) {
     const int na = cur.na, nb = cur.nb;
     int k2 = k + 1;
     SquareUnit nxt;
-    const bool has_next = square_unit(p, k2, nxt);
+    const bool has_next = square_unit<kWin>(p, k2, nxt);
     if (!(ok = wait_one(bar_q, done & 1, wd) && wait_one(full_bar(ug), par_of(ug), wd))) break;
     tc_fence_after_sync();
     if (!early_a) {
@@ -1066,14 +1100,16 @@ __device__ __forceinline__ void mma_role_kv(uint32_t tmem, uint32_t base, uint32
 
 // kD: head dimension. kKV: the kv path (Nq query rows against N keys, the
 // KV range of each head split across CTAs); false: the square problem.
-// kF8 (square problem only): E4M3 Q, K, V and P.
-template <int D, bool kKV, bool kF8 = false, bool kBias = kKV>
+// kF8 (square problem only): E4M3 Q, K, V and P. kBias: the distance bias
+// (applied when p.slopes is set). kWin (square bf16 only): key windows.
+template <int D, bool kKV, bool kF8 = false, bool kBias = kKV, bool kWin = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                           const __grid_constant__ CUtensorMap tmap_k,
                           const __grid_constant__ CUtensorMap tmap_v,
                           const __grid_constant__ CUtensorMap tmap_o, const FwdParams p) {
   static_assert(!(kKV && kF8), "the FP8 path covers the square problem");
+  static_assert(!(kWin && (kKV || kF8)), "kWin selects the windowed square bf16 path");
   using C = Cfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -1142,10 +1178,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t steps = 0;  // this warpgroup's S hand-offs so far (s_full phases)
       uint32_t done = 0;   // work units so far (o_final phases)
       SquareUnit u;
-      for (int k = 0; square_unit(p, k, u); ++k, ++done) {
+      for (int k = 0; square_unit<kWin>(p, k, u); ++k, ++done) {
         const int n = g == 0 ? u.na : u.nb;
-        if (!softmax_role<D, kKV, kF8, kBias>(p, tmem, ctl, u.bh, u.q0, n, g, wd, 0, steps, done & 1,
-                                       &tmap_o, base + C::kStageOff, 2 * done + g))
+        if (!softmax_role<D, kKV, kF8, kBias, kWin>(p, tmem, ctl, u.bh, u.q0, n, g, wd,
+                                                    kWin ? u.j0 : 0, steps, done & 1, &tmap_o,
+                                                    base + C::kStageOff, 2 * done + g))
           break;
         steps += n;
       }
@@ -1156,9 +1193,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsOther<kKV>>();
     if constexpr (!kKV) {
       if (warp == kProducerWarp) {
-        if (lane == 0) producer_role<D, kF8>(&tmap_q, &tmap_k, &tmap_v, base, bars, p, wd);
+        if (lane == 0) producer_role<D, kF8, kWin>(&tmap_q, &tmap_k, &tmap_v, base, bars, p, wd);
       } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_role<D, kF8>(tmem, base, bars, p, wd);
+        if (lane == 0) mma_role<D, kF8, kWin>(tmem, base, bars, p, wd);
       }
     } else {
       const bool alt = p.alt != 0;
@@ -1335,6 +1372,17 @@ int prepare_kernel(int smem_bytes) {
   return status;
 }
 
+// One launch of a square-path instantiation, after its one-time preparation.
+template <auto Kernel>
+int launch_square(unsigned grid, int smem_bytes, cudaStream_t stream, const CUtensorMap& mq,
+                  const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                  const FwdParams& p) {
+  const int prep = prepare_kernel<Kernel>(smem_bytes);
+  if (prep != ATTN_OK) return prep;
+  Kernel<<<grid, kThreads, smem_bytes, stream>>>(mq, mk, mv, mo, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
 // kF8: Q, K, V are E4M3 with the given dequantisation scales (the scores get
 // q_descale * k_descale, O gets v_descale); otherwise bf16 and all scales 1.
 template <int D, bool kF8 = false>
@@ -1367,25 +1415,34 @@ int launch_fused_d(const AttnArgs& a, cudaStream_t stream, float q_descale = 1.0
   p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   p.H = a.H;
   p.slopes = a.slopes;
+  p.wl = a.window_left;
+  p.wr = a.window_right;
   const long long units = static_cast<long long>(p.nqb) * BH;
   if (units > 0x7fffffffLL) return ATTN_ERR_SHAPE;
-  // the distance bias has an instantiation of its own, so that the plain
-  // kernel's exponent loop carries no bias arithmetic
-  constexpr auto plain = fused_attn_fwd_kernel<D, false, kF8, false>;
-  constexpr auto biased = fused_attn_fwd_kernel<D, false, kF8, !kF8>;
-  const bool use_bias = !kF8 && a.slopes != nullptr;
-  const int prep = use_bias ? prepare_kernel<biased>(C::kSmemBytes) : prepare_kernel<plain>(C::kSmemBytes);
-  if (prep != ATTN_OK) return prep;
   // persistent grid: one CTA per SM (one fits), each walking work units in
   // balanced pairs; with no more units than SMs, one unit per CTA (pairing
   // would only put two units behind each other on half the CTAs)
   const int sms = sm_count_current();
   if (sms < 1) return ATTN_ERR_CUDA;
   p.paired = units > sms ? 1 : 0;
-  const long long grid = std::min<long long>(units, sms);
-  (use_bias ? biased : plain)<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(
-      mq, mk, mv, mo, p);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(units, sms));
+  // the distance bias and the key windows have instantiations of their own,
+  // so that the plain kernel's loops carry none of their arithmetic
+  if constexpr (kF8) {
+    return launch_square<fused_attn_fwd_kernel<D, false, true, false>>(grid, C::kSmemBytes, stream,
+                                                                        mq, mk, mv, mo, p);
+  } else {
+    const bool bias = a.slopes != nullptr;
+    if (a.window_left >= 0 || a.window_right >= 0)
+      return bias ? launch_square<fused_attn_fwd_kernel<D, false, false, true, true>>(
+                        grid, C::kSmemBytes, stream, mq, mk, mv, mo, p)
+                  : launch_square<fused_attn_fwd_kernel<D, false, false, false, true>>(
+                        grid, C::kSmemBytes, stream, mq, mk, mv, mo, p);
+    return bias ? launch_square<fused_attn_fwd_kernel<D, false, false, true>>(grid, C::kSmemBytes,
+                                                                             stream, mq, mk, mv, mo, p)
+                : launch_square<fused_attn_fwd_kernel<D, false, false, false>>(
+                      grid, C::kSmemBytes, stream, mq, mk, mv, mo, p);
+  }
 }
 
 // ------------------------------------------------------------ kv path host

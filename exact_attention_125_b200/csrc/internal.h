@@ -20,6 +20,9 @@ struct AttnArgs {
   int causal;
   // per-head linear distance bias slopes (natural-log units), or null
   const float* slopes = nullptr;
+  // key window [i - window_left, i + window_right] around query row i; -1:
+  // unbounded on that side (bf16 path only)
+  int window_left = -1, window_right = -1;
 };
 
 // Fused tcgen05 path (fused_fwd.cu). Arguments already validated.

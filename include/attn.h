@@ -131,8 +131,9 @@ int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
  * normalised fp32 partial O and its lse per range; a second kernel combines
  * them, O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max_s lse_s).
  * With num_splits = 1 the fused kernel writes o and lse directly; when also
- * Nq == Nk (and, for attn_fwd_ext, no window) the call runs attn_fwd's
- * persistent square kernel, with the same results as attn_fwd.
+ * Nq == Nk the call runs attn_fwd's persistent square kernel (for
+ * attn_fwd_ext, its window and bias variants), with the same results as
+ * attn_fwd where no window or bias is asked for.
  *
  * num_splits: 1 .. 256, or 0 for attn_fwd_kv_num_splits(...)'s choice.
  * workspace: device memory of at least

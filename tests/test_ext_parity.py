@@ -37,6 +37,20 @@ CASES = [
     (1, 2, 300, 300, 128, False, -1, -1, "alibi", 1),
     (1, 2, 513, 513, 64, True, -1, -1, "steep", 0),
     (2, 2, 384, 384, 128, False, -1, -1, "steep", 1),
+    # square problems with a window and one split run on the square kernel's
+    # window instantiations: units start at their first row's first key tile;
+    # more units than SMs (paired), one-sided and two-sided windows, a window
+    # wider than N, the diagonal alone, ragged N, both head sizes
+    (2, 40, 700, 700, 128, True, 200, -1, None, 1),
+    (1, 160, 520, 520, 64, True, 300, -1, "alibi", 1),
+    (1, 3, 1000, 1000, 64, False, 100, 300, None, 1),
+    (1, 2, 900, 900, 128, False, 250, 250, "steep", 1),
+    (1, 2, 513, 513, 128, True, 5000, 3, "alibi", 1),
+    (1, 2, 640, 640, 128, False, 129, -1, None, 1),
+    (1, 2, 640, 640, 64, False, -1, 129, "alibi", 1),
+    (1, 2, 384, 384, 128, True, 0, -1, None, 1),
+    # the same square window problem cut into key-range splits (kv path)
+    (1, 2, 300, 300, 128, True, 63, -1, None, 2),
 ]
 
 
@@ -108,6 +122,25 @@ def test_square_ext_without_options_matches_attn_fwd_bit_for_bit(causal):
     o1, l1 = ea.attn_fwd(qg, kg, vg, causal=causal)
     o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=causal, num_splits=1)
     torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("alibi", [False, True])
+@pytest.mark.parametrize("causal", [False, True])
+def test_square_window_over_every_key_matches_unwindowed_bit_for_bit(causal, alibi):
+    # a window wider than the sequence masks nothing: the window
+    # instantiation must then reproduce the unwindowed square kernel exactly
+    # (same tiles, same masks, same arithmetic order)
+    N = 700
+    q, k, v = make_q_kv(1, 3, N, N, 128, seed=23 + int(causal) + 2 * int(alibi))
+    qg, kg, vg = (t.to("cuda") for t in (q, k, v))
+    sl = (torch.tensor([2.0 ** (-8.0 * (h + 1) / 3) for h in range(3)], dtype=torch.float32,
+                       device="cuda") if alibi else None)
+    o1, l1 = ea.attn_fwd_ext(qg, kg, vg, causal=causal, alibi_slopes=sl, num_splits=1)
+    o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=causal, window_left=N, window_right=N,
+                             alibi_slopes=sl, num_splits=1)
+    torch.cuda.synchronize()
+    assert ea.last_device_error() == 0
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
