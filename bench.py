@@ -935,28 +935,44 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
     ws = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step():
+    def step(sl=slopes):
         ea.attn_fwd_ext(q, k, v, o, lse, scale=1.0 / math.sqrt(d), causal=causal, window_left=wl,
-                        window_right=wr, alibi_slopes=slopes, num_splits=splits, workspace=ws,
+                        window_right=wr, alibi_slopes=sl, num_splits=splits, workspace=ws,
                         stream=stream)
+
+    def timed(sl, n):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(n):
+            step(sl)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        return start.elapsed_time(end) / n
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(device)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(device)
+    ms = timed(slopes, steps)
+    # With the bias: the same call without it, timed in alternating samples
+    # with the biased call, so that both see the same clock and power state;
+    # their ratio is the bias's cost.
+    same_run = None
+    if bias:
+        step(None)
+        torch.cuda.synchronize(device)
+        pairs = [(timed(slopes, steps), timed(None, steps)) for _ in range(3)]
+        with_b = statistics.median(a for a, _ in pairs)
+        without = statistics.median(b for _, b in pairs)
+        same_run = {"ms_with_bias": with_b, "ms_without_bias": without,
+                    "with_over_without_throughput": without / with_b,
+                    "samples": f"3 alternating pairs of {steps} launches each"}
     if ea.last_device_error() != 0:
         raise SystemExit(f"device watchdog fired in the line {name}")
-    ms = start.elapsed_time(end) / steps
     flops = 4.0 * B * H * d * costs.ext_visible_pairs(Nq, Nk, causal, wl, wr)
     tf = flops / (ms * 1e-3) / 1e12
     del q, k, v, ws
     torch.cuda.empty_cache()
-    return {"workload": name, "B": B, "H": H, "Nq": Nq, "Nk": Nk, "d": d, "causal": causal,
+    line = {"workload": name, "B": B, "H": H, "Nq": Nq, "Nk": Nk, "d": d, "causal": causal,
             "window_left": wl, "window_right": wr, "distance_bias": bias, "num_splits": splits,
             "ms_per_step": ms, "steps": steps, "tflops": tf, "bound": "tensor",
             "peak_tflops": float(peaks["bf16_tflops"]), "frac": tf / float(peaks["bf16_tflops"]),
@@ -964,6 +980,9 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
                        f"{str(wl >= 0 or wr >= 0).lower()}> (square problem, unsplit)"
                        if Nq == Nk and splits == 1
                        else "fused_attn_fwd_kernel<128, true, false, true, false>")}
+    if same_run is not None:
+        line["against_unbiased_same_run"] = same_run
+    return line
 
 
 def chain_line(device, peaks, rows=65536, cols=8192, steps=10, warmup=3):
