@@ -954,18 +954,23 @@ def ext_line(spec, device, peaks, steps=5, warmup=3):
     torch.cuda.synchronize(device)
     ms = timed(slopes, steps)
     # With the bias: the same call without it, timed in alternating samples
-    # with the biased call, so that both see the same clock and power state;
-    # their ratio is the bias's cost.
+    # with the biased call, each after a 1 s idle gap so that both run below
+    # the power cap at the same clock; their ratio is the bias's cost.
     same_run = None
     if bias:
         step(None)
         torch.cuda.synchronize(device)
-        pairs = [(timed(slopes, steps), timed(None, steps)) for _ in range(3)]
+
+        def gapped(sl):
+            time.sleep(1.0)
+            return timed(sl, steps)
+
+        pairs = [(gapped(slopes), gapped(None)) for _ in range(3)]
         with_b = statistics.median(a for a, _ in pairs)
         without = statistics.median(b for _, b in pairs)
         same_run = {"ms_with_bias": with_b, "ms_without_bias": without,
                     "with_over_without_throughput": without / with_b,
-                    "samples": f"3 alternating pairs of {steps} launches each"}
+                    "samples": f"3 alternating pairs of {steps} launches, each after a 1 s idle gap"}
     if ea.last_device_error() != 0:
         raise SystemExit(f"device watchdog fired in the line {name}")
     flops = 4.0 * B * H * d * costs.ext_visible_pairs(Nq, Nk, causal, wl, wr)

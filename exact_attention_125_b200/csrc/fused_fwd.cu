@@ -352,13 +352,19 @@ __device__ __forceinline__ bool softmax_role(const FwdParams& p, uint32_t tmem, 
     if (kBias && p.slopes) {
       // linear distance bias: x = s * c - slope * log2(e) * |pos - key|
       const float rel = static_cast<float>(row + pos_offset - col0);  // pos - col0
-      const bool left = col0 + kTileRows - 1 <= row_start + pos_offset;   // key <= pos everywhere
+      // key <= pos for every unmasked key of the tile: a tile left of every
+      // row's position, or any tile of a causal problem (the keys past a
+      // row's position are -inf whatever is added to them)
+      const bool left = p.causal || col0 + kTileRows - 1 <= row_start + pos_offset;
       const bool right = col0 >= row_start + kTileRows - 1 + pos_offset;  // key >= pos everywhere
       if ((left || right) && slope_l2 * (kTileRows - 1) <= kBiasBoundSlack) {
         // One side of every row's position: the bias is linear in the
         // column, b(cc) = b0 + dk * cc. The scores stay unbiased here; the
-        // row maximum is bounded by max(s) * c + max(b) and the bias enters
-        // the exponent's FMA (below), one packed add per pair.
+        // row maximum is bounded by max(s) * c + max(b) (max(b) over the
+        // whole tile, masked columns included, so the bound may exceed the
+        // row's largest logit by up to the bias range, at most the slack)
+        // and the bias enters the exponent's FMA (below), one packed add per
+        // pair.
         bias_dk = left ? slope_l2 : -slope_l2;
         bias_b0 = -bias_dk * rel;
         bias_linear = true;

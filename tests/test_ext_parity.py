@@ -51,6 +51,12 @@ CASES = [
     (1, 2, 384, 384, 128, True, 0, -1, None, 1),
     # the same square window problem cut into key-range splits (kv path)
     (1, 2, 300, 300, 128, True, 63, -1, None, 2),
+    # causal with the bias on the square kernel: diagonal tiles take the
+    # linear form too (steep slopes: a bound up to the slack above the row
+    # maximum), ragged N, both head sizes, with and without a window
+    (1, 3, 513, 513, 128, True, -1, -1, "steep", 1),
+    (1, 2, 777, 777, 64, True, -1, -1, "alibi", 1),
+    (1, 2, 640, 640, 128, True, 200, -1, "steep", 1),
 ]
 
 
