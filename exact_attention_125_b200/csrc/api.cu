@@ -9,6 +9,7 @@
 
 #include "../../include/attn.h"
 #include "../../include/chain.h"
+#include "ctx_cache.h"
 #include "internal.h"
 
 namespace {
@@ -64,6 +65,41 @@ attn::AttnArgs pack(const void* q, const void* k, const void* v, void* o, float*
   return a;
 }
 
+// Multiprocessors of the current device, cached per context.
+int sm_count_cached() {
+  static attn::CtxCache<int> cache;
+  int n = 0;
+  if (!cache.get(&n, [](int* out) {
+        int dev = 0;
+        return cudaGetDevice(&dev) == cudaSuccess &&
+               cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
+      }))
+    return 0;
+  return n;
+}
+
+// A square problem whose 256-row work units would fill at most half of the
+// SMs runs as one 128-row query tile per CTA, the layout the split-KV kernel
+// uses for short query ranges: the tile's two softmax warpgroups take
+// alternate KV tiles and merge their (O, m, l) at the end. Twice the CTAs,
+// each with half the KV steps, one launch and no workspace.
+bool small_square(int B, int H, int N) {
+  const int sms = sm_count_cached();
+  const long long units = static_cast<long long>(B) * H * ((N + 255) / 256);
+  return sms > 0 && 2 * units <= sms;
+}
+
+attn::KvPlan query_tile_plan(int N) {
+  attn::KvPlan pl{};
+  pl.T = (N + 127) / 128;
+  pl.tps = pl.T;
+  pl.nsplit = 1;
+  pl.alt = 1;
+  pl.nqb = pl.T;
+  pl.t_begin = 0;
+  return pl;
+}
+
 }  // namespace
 
 extern "C" {
@@ -73,6 +109,11 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   int st = validate(q, k, v, o, lse, B, H, N, d, scale, causal);
   if (st != ATTN_OK) return st;
   if ((st = check_device()) != ATTN_OK) return st;
+  if (small_square(B, H, N)) {
+    attn::AttnKvArgs a{q, k, v, o, lse, B, H, N, N, d, scale, causal, -1, -1, nullptr};
+    return attn::launch_fused_kv(a, query_tile_plan(N), nullptr,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  }
   return attn::launch_fused(pack(q, k, v, o, lse, B, H, N, d, scale, causal),
                             reinterpret_cast<cudaStream_t>(stream));
 }
@@ -146,6 +187,25 @@ int fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, in
     if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   }
   if ((st = check_device()) != ATTN_OK) return st;
+  attn::AttnKvArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.d = d;
+  a.scale = scale;
+  a.causal = causal;
+  a.window_left = window_left;
+  a.window_right = window_right;
+  a.slopes = slopes;
+  if (Nq == Nk && plan.nsplit == 1 && small_square(B, H, Nq))
+    return attn::launch_fused_kv(a, query_tile_plan(Nq), nullptr,
+                                 reinterpret_cast<cudaStream_t>(stream));
   if (Nq == Nk && plan.nsplit == 1) {
     // the square problem, unsplit: the persistent square kernel, which takes
     // the key windows and the distance bias too (the workspace stays unused)
@@ -166,22 +226,6 @@ int fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, in
     s.window_right = window_right;
     return attn::launch_fused(s, reinterpret_cast<cudaStream_t>(stream));
   }
-  attn::AttnKvArgs a;
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.o = o;
-  a.lse = lse;
-  a.B = B;
-  a.H = H;
-  a.Nq = Nq;
-  a.Nk = Nk;
-  a.d = d;
-  a.scale = scale;
-  a.causal = causal;
-  a.window_left = window_left;
-  a.window_right = window_right;
-  a.slopes = slopes;
   return attn::launch_fused_kv(a, plan, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -81,7 +81,12 @@ enum {
  * into swizzled shared memory through an mbarrier ring, tcgen05 MMAs
  * accumulate S = Q K^T and O += P V in tensor memory, and softmax warps keep a
  * running row maximum and row sum (online softmax, exp2 domain). S and P never
- * leave the SM; only O and lse are written.
+ * leave the SM; only O and lse are written. Each CTA works on 256 query rows
+ * at a time; when B*H*ceil(N/256) is at most half the device's SMs, each CTA
+ * takes 128 query rows instead and its two softmax groups split the keys
+ * between them, merging their results at the end (twice the CTAs, no extra
+ * memory). The two layouts agree within floating-point rounding, not bit
+ * for bit.
  *
  * q, k, v (in), o (out): [B, H, N, d] bf16. lse (out): [B, H, N] fp32.
  * Returns ATTN_OK or ATTN_ERR_*; see the conventions above.
@@ -131,9 +136,9 @@ int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
  * normalised fp32 partial O and its lse per range; a second kernel combines
  * them, O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max_s lse_s).
  * With num_splits = 1 the fused kernel writes o and lse directly; when also
- * Nq == Nk the call runs attn_fwd's persistent square kernel (for
- * attn_fwd_ext, its window and bias variants), with the same results as
- * attn_fwd where no window or bias is asked for.
+ * Nq == Nk the call runs what attn_fwd runs for that shape (for
+ * attn_fwd_ext, with its window and bias), with the same results as attn_fwd
+ * where no window or bias is asked for.
  *
  * num_splits: 1 .. 256, or 0 for attn_fwd_kv_num_splits(...)'s choice.
  * workspace: device memory of at least

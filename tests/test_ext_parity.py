@@ -31,16 +31,17 @@ CASES = [
     (1, 2, 700, 700, 128, True, 255, -1, "steep", 0),
     (1, 1, 300, 200, 64, False, 10, 10, None, 1),   # early rows: no key in their window
     (1, 3, 17, 4096, 64, True, 511, -1, "alibi", 0),
-    # square problems without a window run on the persistent square kernel:
-    # non-causal (tiles left of, right of and across the diagonal), steep
-    # slopes (the bias added per logit), d = 64, ragged N
+    # Square problems with one split: with few heads (at most half as many
+    # 256-row units as SMs) they run one 128-row query tile per CTA on the kv
+    # kernel; with many heads (*_SQ below) on the persistent square kernel's
+    # window and bias instantiations. Non-causal (tiles left of, right of and
+    # across the diagonal), steep slopes (the bias added per logit, or a
+    # bound up to the slack above the row maximum), one-sided and two-sided
+    # windows, a window wider than N, the diagonal alone, ragged N, both head
+    # sizes.
     (1, 2, 300, 300, 128, False, -1, -1, "alibi", 1),
     (1, 2, 513, 513, 64, True, -1, -1, "steep", 0),
     (2, 2, 384, 384, 128, False, -1, -1, "steep", 1),
-    # square problems with a window and one split run on the square kernel's
-    # window instantiations: units start at their first row's first key tile;
-    # more units than SMs (paired), one-sided and two-sided windows, a window
-    # wider than N, the diagonal alone, ragged N, both head sizes
     (2, 40, 700, 700, 128, True, 200, -1, None, 1),
     (1, 160, 520, 520, 64, True, 300, -1, "alibi", 1),
     (1, 3, 1000, 1000, 64, False, 100, 300, None, 1),
@@ -51,12 +52,26 @@ CASES = [
     (1, 2, 384, 384, 128, True, 0, -1, None, 1),
     # the same square window problem cut into key-range splits (kv path)
     (1, 2, 300, 300, 128, True, 63, -1, None, 2),
-    # causal with the bias on the square kernel: diagonal tiles take the
-    # linear form too (steep slopes: a bound up to the slack above the row
-    # maximum), ragged N, both head sizes, with and without a window
     (1, 3, 513, 513, 128, True, -1, -1, "steep", 1),
     (1, 2, 777, 777, 64, True, -1, -1, "alibi", 1),
     (1, 2, 640, 640, 128, True, 200, -1, "steep", 1),
+]
+
+# Many heads: the persistent square kernel's window and bias instantiations
+# (more 256-row units than half the SMs; several per CTA where they
+# outnumber the SMs).
+CASES_SQ = [
+    (1, 40, 300, 300, 128, False, -1, -1, "alibi", 1),
+    (1, 40, 384, 384, 128, False, -1, -1, "steep", 1),
+    (1, 40, 1000, 1000, 64, False, 100, 300, None, 1),
+    (1, 40, 900, 900, 128, False, 250, 250, "steep", 1),
+    (1, 40, 513, 513, 128, True, 5000, 3, "alibi", 1),
+    (1, 30, 640, 640, 128, False, 129, -1, None, 1),
+    (1, 30, 640, 640, 64, False, -1, 129, "alibi", 1),
+    (1, 60, 384, 384, 128, True, 0, -1, None, 1),
+    (1, 40, 513, 513, 128, True, -1, -1, "steep", 1),
+    (1, 40, 777, 777, 64, True, -1, -1, "alibi", 1),
+    (1, 40, 640, 640, 128, True, 200, -1, "steep", 1),
 ]
 
 
@@ -68,7 +83,7 @@ def _slopes(kind, H):
     return [0.5 / (h + 1) for h in range(H)]  # steep: a few keys dominate
 
 
-@pytest.mark.parametrize("B,H,Nq,Nk,d,causal,wl,wr,kind,splits", CASES)
+@pytest.mark.parametrize("B,H,Nq,Nk,d,causal,wl,wr,kind,splits", CASES + CASES_SQ)
 def test_ext_all_rows(B, H, Nq, Nk, d, causal, wl, wr, kind, splits):
     _ext_case(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale_of(d))
 
@@ -79,6 +94,8 @@ def test_ext_all_rows(B, H, Nq, Nk, d, causal, wl, wr, kind, splits):
     (1, 2, 100, 1100, 128, True, 300, -1, None, 4),
     (1, 4, 1, 3000, 64, False, -1, -1, "alibi", 3),
     (1, 2, 300, 300, 128, True, -1, -1, "alibi", 1),
+    (1, 40, 300, 300, 128, True, 63, -1, "alibi", 1),
+    (1, 40, 300, 300, 128, False, -1, -1, "steep", 1),
 ])
 def test_ext_zero_and_negative_scale(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale):
     _ext_case(B, H, Nq, Nk, d, causal, wl, wr, kind, splits, scale)
@@ -120,10 +137,11 @@ def test_ext_without_options_matches_attn_fwd_kv_bit_for_bit():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("H", [3, 40])  # the one-tile layout and the 256-row kernel
 @pytest.mark.parametrize("causal", [False, True])
-def test_square_ext_without_options_matches_attn_fwd_bit_for_bit(causal):
-    # Nq == Nk, no window, no bias: the square kernel serves both entry points
-    q, k, v = make_q_kv(1, 3, 700, 700, 128, seed=11 + int(causal))
+def test_square_ext_without_options_matches_attn_fwd_bit_for_bit(causal, H):
+    # Nq == Nk, no window, no bias: both entry points take the same layout
+    q, k, v = make_q_kv(1, H, 700, 700, 128, seed=11 + int(causal))
     qg, kg, vg = (t.to("cuda") for t in (q, k, v))
     o1, l1 = ea.attn_fwd(qg, kg, vg, causal=causal)
     o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=causal, num_splits=1)
@@ -131,16 +149,17 @@ def test_square_ext_without_options_matches_attn_fwd_bit_for_bit(causal):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("H", [3, 40])  # the one-tile layout and the 256-row kernel
 @pytest.mark.parametrize("alibi", [False, True])
 @pytest.mark.parametrize("causal", [False, True])
-def test_square_window_over_every_key_matches_unwindowed_bit_for_bit(causal, alibi):
+def test_square_window_over_every_key_matches_unwindowed_bit_for_bit(causal, alibi, H):
     # a window wider than the sequence masks nothing: the window
-    # instantiation must then reproduce the unwindowed square kernel exactly
-    # (same tiles, same masks, same arithmetic order)
+    # instantiation must then reproduce the unwindowed kernel exactly (same
+    # tiles, same masks, same arithmetic order)
     N = 700
-    q, k, v = make_q_kv(1, 3, N, N, 128, seed=23 + int(causal) + 2 * int(alibi))
+    q, k, v = make_q_kv(1, H, N, N, 128, seed=23 + int(causal) + 2 * int(alibi))
     qg, kg, vg = (t.to("cuda") for t in (q, k, v))
-    sl = (torch.tensor([2.0 ** (-8.0 * (h + 1) / 3) for h in range(3)], dtype=torch.float32,
+    sl = (torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32,
                        device="cuda") if alibi else None)
     o1, l1 = ea.attn_fwd_ext(qg, kg, vg, causal=causal, alibi_slopes=sl, num_splits=1)
     o2, l2 = ea.attn_fwd_ext(qg, kg, vg, causal=causal, window_left=N, window_right=N,

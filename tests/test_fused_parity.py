@@ -15,6 +15,9 @@ from parity_util import (check_against_oracle, empty_outputs, sampled, scale_of,
 
 pytestmark = pytest.mark.gpu
 
+# With at most half as many 256-row work units as SMs, attn_fwd runs one
+# 128-row query tile per CTA (its two softmax groups split the keys): these
+# shapes check that layout.
 SMALL = [
     # B, H, N, d, causal
     (1, 1, 128, 64, False),
@@ -58,6 +61,26 @@ MANY_UNITS = [
     (2, 40, 700, 64, False),
     (1, 80, 1100, 128, True),
 ]
+
+
+# The same edge cases (one key, two keys, a ragged last tile, a query tile b
+# past N) with enough heads that the persistent 256-row kernel runs them.
+SQUARE_EDGES = [
+    # B, H, N, d, causal
+    (1, 160, 1, 64, False),
+    (1, 160, 2, 128, True),
+    (1, 80, 127, 64, True),
+    (1, 80, 129, 128, False),
+    (1, 80, 257, 64, True),
+    (2, 40, 255, 128, False),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", SQUARE_EDGES)
+def test_square_kernel_edges_all_rows(B, H, N, d, causal):
+    q, k, v = make_qkv(B, H, N, d, seed=7 * N + H + d + int(causal))
+    o, lse = _run(q, k, v, scale_of(d), causal)
+    check_against_oracle(q, k, v, o, lse, scale_of(d), causal, what=f"{(B, H, N, d, causal)}")
 
 
 @pytest.mark.parametrize("B,H,N,d,causal", MANY_UNITS)
@@ -148,12 +171,13 @@ def test_outputs_do_not_depend_on_stale_memory():
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
 
 
+@pytest.mark.parametrize("H", [2, 80])  # the one-tile layout and the 256-row kernel
 @pytest.mark.parametrize("scale", [0.0, -0.125, -1.0])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d", [64, 128])
-def test_zero_and_negative_scale(d, causal, scale):
+def test_zero_and_negative_scale(d, causal, scale, H):
     # any finite scale is accepted; a negative one favours the smallest q.k
-    q, k, v = make_qkv(1, 2, 333, d, seed=31 + d + int(causal))
+    q, k, v = make_qkv(1, H, 333, d, seed=31 + d + int(causal))
     o, lse = _run(q, k, v, scale, causal)
     check_against_oracle(q, k, v, o, lse, scale, causal, what=f"scale {scale}, d {d}")
     if scale == 0.0:
