@@ -261,9 +261,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // in for 0 when x = -inf); relative error <= kExp2PolyMaxRelErr + fp32 rounding.
 // So a masked logit (-inf) on these columns gives a weight of 2^-125, not 0.
 // The callers rely on what follows: a row's sum l >= 1 once it has seen an
-// allowed key (2^-125 is then lost in fp32 rounding of l and of O), and a row
-// that has seen none (m = -inf, only possible in a split of the kv path) has
-// its l reset to 0 before the epilogue, which writes O = 0 and lse = -inf.
+// allowed key (2^-125 is then lost in fp32 rounding of l and of O). A row
+// that has seen none so far (m = -inf: a leading KV tile wholly outside its
+// key window, or a split of the kv path) carries only such weights; its first
+// allowed key raises m from -inf, and the rescale by alpha = 2^-inf = 0
+// clears l and the O row exactly. A row that never sees one (only possible
+// in a split of the kv path) has its l reset to 0 before the epilogue, which
+// writes O = 0 and lse = -inf, and the two-warpgroup merge of the kv path
+// gives a side with m = -inf the weight 0.
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -125.0f);
   const float t = __fadd_rn(x, 12582912.0f);
